@@ -1,0 +1,165 @@
+/*
+ * moga.h -- C ABI of the B200 (sm_100a) MoGA visual-attention layer forward.
+ *
+ * The layer (MoGA paper: papernotes.org ICLR 2026 note, flowchart and key
+ * designs 1-4; jxzklqfsx.com translation, section 方法) is:
+ *
+ *   route    r = x . W_r, p = softmax(r), g = argmax p, gate = p[g]
+ *   permute  tokens grouped by g (stable), cu_seqlens / counts / max_seqlen
+ *   MoGA     o_moga[t] = gate[t] * SA(q_t, K_g(t), V_g(t))   (scattered back)
+ *   STGA     o_win[t]  = SA over the token's spatial window x temporal group,
+ *                        K/V widened by frames of the adjacent shot at a cut
+ *            o_frame[t]= SA over the token's latent frame
+ *   mean     out = (o_moga + o_win + o_frame) / 3
+ *   loss     L_gb = alpha * M * sum_i F_i * P_i
+ *
+ * Conventions for every call:
+ *   - Pointers are DEVICE pointers unless marked HOST.  The caller allocates
+ *     and owns every buffer, including workspaces; the library allocates and
+ *     frees nothing.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream) and never synchronise the host.
+ *   - Tensors are dense row-major.  Q, K, V and outputs use the token-major
+ *     "thd" layout [N][H][hd] (bf16 Q/K/V, fp32 accumulator).
+ *   - Arguments are validated before any launch.  A bad argument returns
+ *     MOGA_ERR_INVALID_ARG (or MOGA_ERR_UNSUPPORTED / MOGA_ERR_WORKSPACE) and
+ *     launches nothing; moga_last_error() then describes it.  A failed launch
+ *     returns MOGA_ERR_CUDA.  Kernels never trap: a device-side wait that
+ *     runs out of time records MOGA_ERR_TIMEOUT in a per-device error word,
+ *     which moga_device_status() reports.
+ *   - Limits: N * H < 2^31, 1 <= M <= 32, d % 8 == 0, hd in {64, 128}.
+ */
+#ifndef MOGA_H
+#define MOGA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOGA_OK = 0,
+  MOGA_ERR_INVALID_ARG = 1,
+  MOGA_ERR_UNSUPPORTED = 2,
+  MOGA_ERR_WORKSPACE = 3,
+  MOGA_ERR_CUDA = 4,
+  MOGA_ERR_TIMEOUT = 5
+} moga_status;
+
+typedef enum { MOGA_F32 = 0, MOGA_BF16 = 1 } moga_dtype;
+
+/* Static-group geometry (note, key design 4; translation, 时空分组注意力).
+ * Tokens are in raster order t = frame*h*w + row*w + col.  Windows tile the
+ * frame without overlap (h % win_h == 0, w % win_w == 0).  Each shot is cut
+ * into ceil(len / tg_max) temporal groups of as-equal-as-possible length,
+ * longer first (tg_max == 0: one group per shot).  A group that starts a shot
+ * after a cut adds the last min(aug_frames, len) frames of the previous shot
+ * to its keys/values; a group that ends a shot before a cut adds the first
+ * min(aug_frames, len) frames of the next shot.  Queries are never added. */
+typedef struct {
+  int32_t T, h, w;           /* latent frames, token rows and columns per frame */
+  int32_t win_h, win_w;      /* spatial window */
+  int32_t n_shots;           /* >= 1 */
+  const int32_t* shot_len;   /* HOST [n_shots], each >= 1, summing to T */
+  int32_t tg_max;            /* max frames per temporal group, 0 = whole shot */
+  int32_t aug_frames;        /* frames borrowed from each adjacent shot (pages: 2) */
+} moga_stga_geom;
+
+/* ---------------------------------------------------------------- routing --
+ * Linear top-1 router (note, key design 1; blog section 2.3):
+ *   r = x . W_r (+ bias), p = softmax(r), g = argmax_i p_i (lowest index on
+ *   a tie), gate_prob = p_g.  Logits are accumulated in fp32.
+ * x:         [N][d], dtype `dt` (MOGA_F32 or MOGA_BF16)
+ * w_r:       [d][M], same dtype as x
+ * bias:      [M] fp32 or NULL (the pages' router has no bias)
+ * group_id:  [N] int32 out;  gate_prob: [N] fp32 out
+ * ws:        workspace of at least moga_route_ws_bytes(N, M) bytes; on return
+ *            it holds per-block partial sums of p(i|x) that
+ *            moga_balance_loss() reads.  Keep it until the loss is taken.
+ */
+size_t moga_route_ws_bytes(int64_t N, int32_t M);
+moga_status moga_route(const void* x, const void* w_r, moga_dtype dt, const float* bias,
+                       int64_t N, int32_t d, int32_t M,
+                       int32_t* group_id, float* gate_prob,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- permute --
+ * Stable counting sort of tokens by group (note, key design 2: permute so
+ * each group is contiguous; boundaries as cu_seqlens / max_seqlen):
+ *   counts[i] = #{t : g_t = i}, cu_seqlens = exclusive prefix (cu[M] = N),
+ *   perm[cu[i] + j] = the j-th smallest token index with g = i,
+ *   *max_seqlen = max_i counts[i].
+ * group_id: [N] int32, every value in [0, M) (values outside are not checked
+ *           on the host; the kernels skip them and the result is then
+ *           undefined)
+ * perm [N], cu_seqlens [M+1], counts [M], max_seqlen [1]: int32 out
+ * ws:       at least moga_permute_ws_bytes(N, M) bytes of scratch.
+ */
+size_t moga_permute_ws_bytes(int64_t N, int32_t M);
+moga_status moga_permute(const int32_t* group_id, int64_t N, int32_t M,
+                         int32_t* perm, int32_t* cu_seqlens, int32_t* counts, int32_t* max_seqlen,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* -------------------------------------------------------- group attention --
+ * MoGA attention (note, key designs 1-2): for every group i and head h,
+ * full non-causal softmax attention among the tokens perm[cu[i] .. cu[i+1]),
+ * each output row scaled by its token's gate and written to that token's own
+ * row:  o_acc[perm[j]][h][:] = gate_prob[perm[j]] * softmax(q k^T * scale) v.
+ * q, k, v:  [N][H][hd] bf16;  perm, cu_seqlens: from moga_permute
+ * o_acc:    [N][H][hd] fp32, OVERWRITTEN for every token (empty groups are
+ *           skipped; tokens are covered because perm is a permutation)
+ * softmax_scale: usually 1/sqrt(hd).
+ */
+moga_status moga_group_attn(const void* q, const void* k, const void* v,
+                            int64_t N, int32_t H, int32_t hd,
+                            const int32_t* perm, const int32_t* cu_seqlens, int32_t M,
+                            const float* gate_prob, float softmax_scale,
+                            float* o_acc, void* stream);
+
+/* ------------------------------------------------------------------- STGA --
+ * Static spatial-temporal group attention plus per-frame attention (note,
+ * key design 4; translation, 时空分组注意力; blog 3.2): for every token,
+ *   o_acc[t] += SA(q_t, K/V of its window group incl. adjacent-shot frames)
+ *             + SA(q_t, K/V of its latent frame).
+ * q, k, v: [N][H][hd] bf16 with N = T*h*w;  o_acc: [N][H][hd] fp32, ADDED TO.
+ * geom: HOST pointer, read during the call only.
+ */
+moga_status stga_attn(const void* q, const void* k, const void* v, int32_t H, int32_t hd,
+                      const moga_stga_geom* geom, float softmax_scale,
+                      float* o_acc, void* stream);
+
+/* ------------------------------------------------------------------- mean --
+ * Three-way mean (note, flowchart "多组输出取均值" and key design 4):
+ *   out[i] = bf16_rn(o_acc[i] / 3) for i < n_elems, where o_acc already
+ *   holds o_moga + o_win + o_frame.
+ * o_acc: fp32 [n_elems];  out: bf16 [n_elems] (16-byte aligned pointers).
+ */
+moga_status visual_attn_mean(const float* o_acc, int64_t n_elems, void* out, void* stream);
+
+/* ------------------------------------------------------------------- loss --
+ * Group-balancing loss (note, key design 3):
+ *   L_gb = alpha * M * sum_i F_i * P_i,  F_i = counts[i] / N,
+ *   P_i = (1/N) sum_t p(i | x_t)   (mean over all N tokens).
+ * counts: [M] int32 from moga_permute;  route_ws: the workspace moga_route
+ * filled for the same N and M;  loss: [1] fp64 out (device).
+ */
+moga_status moga_balance_loss(const int32_t* counts, const void* route_ws, int64_t N, int32_t M,
+                              float alpha, double* loss, void* stream);
+
+/* ------------------------------------------------------------- diagnostics */
+/* Text of the last host-side error of the calling thread ("" if none). */
+const char* moga_last_error(void);
+/* Synchronises `stream`, then reads and clears the current device's error
+ * word: MOGA_OK, or the first device-side error recorded since the last
+ * call (e.g. MOGA_ERR_TIMEOUT from a bounded wait). */
+moga_status moga_device_status(void* stream);
+/* Library version string. */
+const char* moga_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOGA_H */

@@ -1,0 +1,168 @@
+"""MoGA visual-attention layer forward on B200 (sm_100a).
+
+Thin Python face of libmoga.so (include/moga.h).  Tensors are torch CUDA
+tensors; torch supplies device memory and the current stream, the library's
+kernels do every step of the layer:
+
+    g, gate, ws = moga_route(x, w_r, bias)          # linear top-1 router
+    perm, cu, counts, maxlen = moga_permute(g, M)   # stable group permute
+    o = moga_group_attn(q, k, v, perm, cu, gate, M) # MoGA groups (o = ...)
+    stga_attn(q, k, v, geom, o_acc=o)               # windows + frames (o += ...)
+    out = visual_attn_mean(o)                       # bf16 (o / 3)
+    loss = moga_balance_loss(counts, ws, N, M, a)   # L_gb (fp64 scalar)
+
+`visual_attention_forward` chains the six calls.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+
+import torch
+
+from ._lib import MOGA_BF16, MOGA_F32, MogaError, StgaGeom, check, lib  # noqa: F401
+
+__all__ = ["moga_route", "moga_permute", "moga_group_attn", "stga_attn", "visual_attn_mean",
+           "moga_balance_loss", "visual_attention_forward", "device_status", "MogaError", "geom_struct"]
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need(t, dtype, name, dim=None):
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dim is not None and t.dim() != dim:
+        raise ValueError("%s must have %d dims" % (name, dim))
+
+
+def moga_route(x: torch.Tensor, w_r: torch.Tensor, bias: torch.Tensor | None = None):
+    """r = x W_r (+bias), p = softmax(r), g = argmax p.  Returns (g int32 [N], gate fp32 [N], ws)."""
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("x must be float32 or bfloat16")
+    _need(x, x.dtype, "x", 2)
+    _need(w_r, x.dtype, "w_r", 2)
+    N, d = x.shape
+    M = w_r.shape[1]
+    if w_r.shape[0] != d:
+        raise ValueError("w_r must be [d, M]")
+    if bias is not None:
+        _need(bias, torch.float32, "bias", 1)
+    L = lib()
+    ws_bytes = L.moga_route_ws_bytes(N, M)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=x.device)
+    g = torch.empty(N, dtype=torch.int32, device=x.device)
+    gate = torch.empty(N, dtype=torch.float32, device=x.device)
+    dt = MOGA_BF16 if x.dtype == torch.bfloat16 else MOGA_F32
+    check(L.moga_route(_ptr(x), _ptr(w_r), dt, _ptr(bias), N, d, M, _ptr(g), _ptr(gate), _ptr(ws), ws.numel(),
+                       _stream()), "moga_route")
+    return g, gate, ws
+
+
+def moga_permute(group_id: torch.Tensor, M: int):
+    """Stable group permute.  Returns (perm [N], cu_seqlens [M+1], counts [M], max_seqlen [1]), int32."""
+    _need(group_id, torch.int32, "group_id", 1)
+    N = group_id.shape[0]
+    L = lib()
+    ws_bytes = L.moga_permute_ws_bytes(N, M)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=group_id.device)
+    dev = group_id.device
+    perm = torch.empty(N, dtype=torch.int32, device=dev)
+    cu = torch.empty(M + 1, dtype=torch.int32, device=dev)
+    counts = torch.empty(M, dtype=torch.int32, device=dev)
+    mx = torch.empty(1, dtype=torch.int32, device=dev)
+    check(L.moga_permute(_ptr(group_id), N, M, _ptr(perm), _ptr(cu), _ptr(counts), _ptr(mx), _ptr(ws), ws.numel(),
+                         _stream()), "moga_permute")
+    return perm, cu, counts, mx
+
+
+def _check_qkv(q, k, v):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, torch.bfloat16, name, 3)
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k, v must share the shape [N, H, hd]")
+    return q.shape
+
+
+def moga_group_attn(q, k, v, perm, cu_seqlens, gate_prob, M: int, softmax_scale: float | None = None,
+                    o_acc: torch.Tensor | None = None):
+    """o_acc[perm[j]] = gate * softmax(q k^T * scale) v inside each group (written, fp32)."""
+    N, H, hd = _check_qkv(q, k, v)
+    _need(perm, torch.int32, "perm", 1)
+    _need(cu_seqlens, torch.int32, "cu_seqlens", 1)
+    _need(gate_prob, torch.float32, "gate_prob", 1)
+    if o_acc is None:
+        o_acc = torch.empty((N, H, hd), dtype=torch.float32, device=q.device)
+    _need(o_acc, torch.float32, "o_acc", 3)
+    scale = 1.0 / math.sqrt(hd) if softmax_scale is None else softmax_scale
+    check(lib().moga_group_attn(_ptr(q), _ptr(k), _ptr(v), N, H, hd, _ptr(perm), _ptr(cu_seqlens), M,
+                                _ptr(gate_prob), scale, _ptr(o_acc), _stream()), "moga_group_attn")
+    return o_acc
+
+
+def geom_struct(geom: dict):
+    """C geometry struct from a dict(T, h, w, win_h, win_w, shots, tg_max, aug); keeps the shot array alive."""
+    shots = (ctypes.c_int32 * len(geom["shots"]))(*geom["shots"])
+    s = StgaGeom(geom["T"], geom["h"], geom["w"], geom["win_h"], geom["win_w"], len(geom["shots"]),
+                 ctypes.cast(shots, ctypes.POINTER(ctypes.c_int32)), geom["tg_max"], geom["aug"])
+    return s, shots
+
+
+def stga_attn(q, k, v, geom: dict, softmax_scale: float | None = None, o_acc: torch.Tensor | None = None):
+    """o_acc += window-group attention + per-frame attention (fp32)."""
+    N, H, hd = _check_qkv(q, k, v)
+    if o_acc is None:
+        o_acc = torch.zeros((N, H, hd), dtype=torch.float32, device=q.device)
+    _need(o_acc, torch.float32, "o_acc", 3)
+    scale = 1.0 / math.sqrt(hd) if softmax_scale is None else softmax_scale
+    s, keep = geom_struct(geom)
+    check(lib().stga_attn(_ptr(q), _ptr(k), _ptr(v), H, hd, ctypes.byref(s), scale, _ptr(o_acc), _stream()),
+          "stga_attn")
+    del keep
+    return o_acc
+
+
+def visual_attn_mean(o_acc: torch.Tensor, out: torch.Tensor | None = None):
+    """out = bf16(o_acc / 3)."""
+    _need(o_acc, torch.float32, "o_acc")
+    if out is None:
+        out = torch.empty(o_acc.shape, dtype=torch.bfloat16, device=o_acc.device)
+    _need(out, torch.bfloat16, "out")
+    check(lib().visual_attn_mean(_ptr(o_acc), o_acc.numel(), _ptr(out), _stream()), "visual_attn_mean")
+    return out
+
+
+def moga_balance_loss(counts, route_ws, N: int, M: int, alpha: float, loss: torch.Tensor | None = None):
+    """L_gb = alpha * M * sum_i F_i P_i as a fp64 device scalar."""
+    _need(counts, torch.int32, "counts", 1)
+    if loss is None:
+        loss = torch.empty(1, dtype=torch.float64, device=counts.device)
+    check(lib().moga_balance_loss(_ptr(counts), _ptr(route_ws), N, M, alpha, _ptr(loss), _stream()),
+          "moga_balance_loss")
+    return loss
+
+
+def device_status():
+    """Synchronises the current stream and raises if a kernel recorded a device-side error."""
+    check(lib().moga_device_status(_stream()), "moga_device_status")
+
+
+def visual_attention_forward(x, w_r, bias, q, k, v, M: int, geom: dict, alpha: float,
+                             softmax_scale: float | None = None):
+    """The whole layer: returns dict(out bf16 [N,H,hd], loss fp64 [1], g, gate, perm, cu_seqlens, counts)."""
+    g, gate, ws = moga_route(x, w_r, bias)
+    perm, cu, counts, mx = moga_permute(g, M)
+    o = moga_group_attn(q, k, v, perm, cu, gate, M, softmax_scale)
+    stga_attn(q, k, v, geom, softmax_scale, o_acc=o)
+    out = visual_attn_mean(o)
+    loss = moga_balance_loss(counts, ws, x.shape[0], M, alpha)
+    return dict(out=out, loss=loss, g=g, gate=gate, perm=perm, cu_seqlens=cu, counts=counts, max_seqlen=mx)

@@ -1,0 +1,28 @@
+// Shared device/host helpers of the MoGA sm_100a library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/moga.h"
+
+namespace moga {
+
+// Host: record an error message for moga_last_error() and return `st`.
+moga_status fail(moga_status st, const char* fmt, ...);
+// Host: map the last launch error to MOGA_ERR_CUDA (with message) or MOGA_OK.
+moga_status check_launch(const char* what);
+
+// Device error word (one per device, lazily created by the CUDA runtime).
+// The library is built as one translation unit (moga_lib.cu), so the word is
+// defined here once.
+__device__ int g_device_error = 0;
+
+__device__ __forceinline__ void record_device_error(int code) {
+  atomicCAS(&g_device_error, 0, code);
+}
+
+__host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace moga

@@ -1,0 +1,7 @@
+// Single translation unit of the MoGA sm_100a library (one device error word,
+// no relocatable device code needed).
+#include "api_common.cu"
+#include "route.cu"
+#include "permute.cu"
+#include "mean_loss.cu"
+#include "attention.cu"

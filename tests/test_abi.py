@@ -1,0 +1,111 @@
+"""The C ABI library loads, exports every declared symbol and validates arguments on the host (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_attention_long_moga_b200 import _lib
+from sparse_attention_long_moga_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moga.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return _lib.load()
+
+
+def declared_functions(path=HEADER):
+    text = open(path).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:moga_status|size_t|const char\s*\*|void)\s+(\w+)\s*\(", text, flags=re.M)
+
+
+def test_header_declares_the_six_calls():
+    names = declared_functions()
+    for n in ("moga_route", "moga_permute", "moga_group_attn", "stga_attn", "visual_attn_mean",
+              "moga_balance_loss"):
+        assert n in names
+    assert set(names) == set(_lib.SIGNATURES)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_workspace_sizes(lib):
+    assert lib.moga_route_ws_bytes(0, 5) == 0
+    assert lib.moga_route_ws_bytes(1000, 33) == 0
+    assert lib.moga_route_ws_bytes(32760, 5) == 256 * 5 * 4
+    assert lib.moga_permute_ws_bytes(32760, 5) == 2 * 16 * 5 * 4
+    assert lib.moga_permute_ws_bytes(-1, 5) == 0
+
+
+FAKE = ctypes.c_void_p(4096)   # never dereferenced: validation fails first
+
+
+def test_route_argument_checks(lib):
+    st = lib.moga_route(None, FAKE, 1, None, 10, 8, 4, FAKE, FAKE, FAKE, 4096, None)
+    assert st == 1 and b"null" in lib.moga_last_error()
+    assert lib.moga_route(FAKE, FAKE, 1, None, 10, 8, 33, FAKE, FAKE, FAKE, 4096, None) == 1
+    assert lib.moga_route(FAKE, FAKE, 1, None, 10, 12, 4, FAKE, FAKE, FAKE, 4096, None) == 1   # d % 8
+    assert lib.moga_route(FAKE, FAKE, 7, None, 10, 8, 4, FAKE, FAKE, FAKE, 4096, None) == 1    # dtype
+    assert lib.moga_route(FAKE, FAKE, 1, None, 0, 8, 4, FAKE, FAKE, FAKE, 4096, None) == 1     # N
+    assert lib.moga_route(FAKE, FAKE, 1, None, 1000, 8, 4, FAKE, FAKE, FAKE, 4, None) == 3     # workspace
+
+
+def test_permute_argument_checks(lib):
+    assert lib.moga_permute(FAKE, 100, 0, FAKE, FAKE, FAKE, FAKE, FAKE, 4096, None) == 1
+    assert lib.moga_permute(FAKE, 100000, 8, FAKE, FAKE, FAKE, FAKE, FAKE, 8, None) == 3
+    assert lib.moga_permute(None, 100, 4, FAKE, FAKE, FAKE, FAKE, FAKE, 4096, None) == 1
+
+
+def test_attention_argument_checks(lib):
+    assert lib.moga_group_attn(FAKE, FAKE, FAKE, 100, 2, 96, FAKE, FAKE, 4, FAKE, 0.1, FAKE, None) == 2
+    assert b"head_dim" in lib.moga_last_error()
+    assert lib.moga_group_attn(FAKE, FAKE, FAKE, 100, 2, 128, FAKE, FAKE, 40, FAKE, 0.1, FAKE, None) == 1
+    assert lib.moga_group_attn(FAKE, FAKE, FAKE, 100, 2, 128, FAKE, FAKE, 4, FAKE, -1.0, FAKE, None) == 1
+    assert lib.moga_group_attn(FAKE, FAKE, FAKE, 1 << 30, 4, 128, FAKE, FAKE, 4, FAKE, 0.1, FAKE, None) == 1
+    mis = ctypes.c_void_p(4096 + 8)
+    assert lib.moga_group_attn(mis, FAKE, FAKE, 100, 2, 128, FAKE, FAKE, 4, FAKE, 0.1, FAKE, None) == 1
+
+
+def _geom(**kw):
+    g = dict(T=4, h=4, w=4, win_h=2, win_w=2, shots=[2, 2], tg_max=0, aug=2)
+    g.update(kw)
+    return g
+
+
+@pytest.mark.parametrize("bad,msg", [
+    (dict(shots=[2, 1]), b"sum"),
+    (dict(win_h=3), b"tile"),
+    (dict(shots=[4, 0], T=4), b"length"),
+    (dict(tg_max=-1), b"geometry"),
+])
+def test_stga_geometry_checks(lib, bad, msg):
+    s, keep = _geom_struct(_geom(**bad))
+    st = lib.stga_attn(FAKE, FAKE, FAKE, 2, 128, ctypes.byref(s), 0.1, FAKE, None)
+    assert st == 1 and msg in lib.moga_last_error(), lib.moga_last_error()
+
+
+def _geom_struct(g):
+    shots = (ctypes.c_int32 * len(g["shots"]))(*g["shots"])
+    s = _lib.StgaGeom(g["T"], g["h"], g["w"], g["win_h"], g["win_w"], len(g["shots"]),
+                      ctypes.cast(shots, ctypes.POINTER(ctypes.c_int32)), g["tg_max"], g["aug"])
+    return s, shots
+
+
+def test_mean_and_loss_argument_checks(lib):
+    assert lib.visual_attn_mean(None, 10, FAKE, None) == 1
+    assert lib.visual_attn_mean(FAKE, 0, FAKE, None) == 1
+    assert lib.visual_attn_mean(ctypes.c_void_p(4100), 10, FAKE, None) == 1
+    assert lib.moga_balance_loss(FAKE, FAKE, 10, 0, 0.1, FAKE, None) == 1
+    assert lib.moga_balance_loss(None, FAKE, 10, 4, 0.1, FAKE, None) == 1
+
+
+def test_version(lib):
+    assert b"sm_100a" in lib.moga_version()

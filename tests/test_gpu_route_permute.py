@@ -1,0 +1,81 @@
+"""GPU parity: router, permute and balance loss against the fp64 oracle.
+
+Group ids, perm, cu_seqlens, counts and max_seqlen must be bit-exact (inputs
+carry a top-2 routing margin of at least 1e-3); gate probabilities agree to a
+relative 1e-5 (fp32 softmax of M values); L_gb to a relative 1e-5.
+"""
+import numpy as np
+import pytest
+
+from _data import GATE_REL, LOSS_REL, Case
+from oracle import layer as olayer
+from oracle import permute as opermute
+from synth import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+EDGE = W.Workload("edge_300", T=5, h=6, w=10, d=64, H=3, hd=128, M=7, shots=(2, 1, 2), tg_max=2,
+                  win_h=3, win_w=5)
+
+CASES = {
+    "tiny": W.TINY,
+    "wan13b_5s": W.WAN13B_5S,
+    "multishot_skewed": W.MULTISHOT_10S,
+    "edge_M7_N300": EDGE,
+    "edge_M1": EDGE.with_(name="edge_M1", M=1),
+    "edge_M32": EDGE.with_(name="edge_M32", M=32, T=7, shots=(3, 4)),
+    "edge_N1": W.Workload("edge_N1", T=1, h=1, w=1, d=16, H=1, hd=64, M=3, shots=(1,), tg_max=0,
+                          win_h=1, win_w=1),
+    "edge_f32_ragged": W.Workload("edge_f32", T=3, h=7, w=9, d=24, H=1, hd=64, M=5, shots=(3,), tg_max=0,
+                                  win_h=7, win_w=9, x_dtype="f32"),
+}
+
+
+@pytest.fixture(scope="module", params=sorted(CASES))
+def routed(request, cuda_device):
+    import sparse_attention_long_moga_b200 as moga
+    case = Case(CASES[request.param], with_qkv=False)
+    t = case.gpu()
+    g, gate, ws = moga.moga_route(t["x"], t["w_r"], t["bias"])
+    M = case.wl.M
+    perm, cu, counts, mx = moga.moga_permute(g, M)
+    loss = moga.moga_balance_loss(counts, ws, case.wl.N, M, case.wl.alpha)
+    moga.device_status()
+    return case, dict(g=g.cpu().numpy(), gate=gate.cpu().numpy(), perm=perm.cpu().numpy(), cu=cu.cpu().numpy(),
+                      counts=counts.cpu().numpy(), mx=int(mx.item()), loss=float(loss.item()))
+
+
+def test_group_ids_bit_exact(routed):
+    case, got = routed
+    g, p_g, p = case.route64()
+    assert np.array_equal(got["g"], g.astype(np.int32))
+
+
+def test_gate_prob(routed):
+    case, got = routed
+    g, p_g, p = case.route64()
+    np.testing.assert_allclose(got["gate"], p_g, rtol=GATE_REL, atol=0)
+
+
+def test_permute_bit_exact(routed):
+    case, got = routed
+    g, _, _ = case.route64()
+    perm, cu, counts, mx = opermute.permute(g, case.wl.M)
+    assert np.array_equal(got["perm"], perm.astype(np.int32))
+    assert np.array_equal(got["cu"], cu.astype(np.int32))
+    assert np.array_equal(got["counts"], counts.astype(np.int32))
+    assert got["mx"] == mx
+
+
+def test_balance_loss(routed):
+    case, got = routed
+    g, _, p = case.route64()
+    counts = np.bincount(g, minlength=case.wl.M)
+    ref = olayer.balance_loss(counts, p, case.wl.alpha)
+    assert got["loss"] == pytest.approx(ref, rel=LOSS_REL)
+
+
+def test_skewed_router_fraction(cuda_device):
+    case = Case(W.MULTISHOT_10S, with_qkv=False)
+    g, _, _ = case.route64()
+    assert 0.395 <= np.mean(g == 0) <= 0.405
