@@ -1,0 +1,380 @@
+#!/usr/bin/env python
+"""Benchmark: MoGA visual-attention layer forward (route, permute, MoGA group
+attention, STGA window + frame attention, three-way mean, balance loss) on
+synthetic Wan-1.3B-shaped latents: 21 frames x 30 x 52 = 32,760 tokens,
+d = 1536, 12 heads x 128, M = 5, one shot, temporal groups of <= 7 frames,
+15 x 26 windows.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one full layer forward over one sequence, inputs resident in HBM.
+Between timed steps a 256 MiB buffer is written to flush L2 (outside the
+timed events).  Under torchrun each rank runs its own sequence (independent
+problems, no data-path collective); the job time is the max over ranks.
+`--impl reference` times the fp64 CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from synth import workloads as W  # noqa: E402
+
+METRIC = "visual-attn layer fwd tokens/s (bf16); group-attn % of tcgen05 bf16 peak"
+WORKLOAD = W.WAN13B_5S
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except OSError:
+        return PEAKS_FALLBACK, "fallback"
+
+
+def moga_flops(counts, H, hd):
+    return 4.0 * H * hd * float(np.sum(np.asarray(counts, dtype=np.float64) ** 2))
+
+
+def stga_flops(wl):
+    """4*H*hd*(sum over window groups n_q*n_kv + T*(hw)^2), from the geometry (readings of the pages)."""
+    whw = wl.win_h * wl.win_w
+    n_win = (wl.h // wl.win_h) * (wl.w // wl.win_w)
+    tot = 0.0
+    for s, L in enumerate(wl.shots):
+        n = 1 if wl.tg_max == 0 else -(-L // wl.tg_max)
+        q, r = divmod(L, n)
+        for i in range(n):
+            run = q + (1 if i < r else 0)
+            kv = run
+            if i == 0 and s > 0:
+                kv += min(wl.aug, wl.shots[s - 1])
+            if i == n - 1 and s + 1 < len(wl.shots):
+                kv += min(wl.aug, wl.shots[s + 1])
+            tot += n_win * (run * whw) * (kv * whw)
+    tot += wl.T * float(wl.hw) ** 2
+    return 4.0 * wl.H * wl.hd * tot
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def make_inputs(wl):
+    """Seeded synthetic inputs (stored margin redraws applied), as numpy stored values."""
+    redraw = W.redraw_map(wl)
+    x = W.x_stored(wl, redraw)
+    w = W.w_r_stored(wl)
+    q, k, v = (W.qkv_stored(wl, n, redraw) for n in ("q", "k", "v"))
+    return dict(x=x, w_r=w, q=q, k=k, v=v)
+
+
+# ----------------------------------------------------------------------------- CPU oracle arm
+
+def oracle_sample(wl, inputs, heads=(0,)):
+    """Times the fp64 oracle as it stands: route + permute + loss over all N
+    tokens, then the MoGA, window and frame attention and the mean over all N
+    tokens for the listed heads.  Returns (tokens/s extrapolated to all heads,
+    details)."""
+    from oracle import attention as oatt
+    from oracle import layer as olayer
+    from oracle import permute as opermute
+    from oracle import route as oroute
+    from oracle import stga as ostga
+
+    x = W.bf16_bits_to_f64(inputs["x"]) if inputs["x"].dtype == np.uint16 else inputs["x"].astype(np.float64)
+    w = W.bf16_bits_to_f64(inputs["w_r"]) if inputs["w_r"].dtype == np.uint16 else inputs["w_r"].astype(np.float64)
+    t0 = time.perf_counter()
+    g, p_g, p = oroute.route(x, w, W.bias_f64(wl))
+    perm, cu, counts, mx = opermute.permute(g, wl.M)
+    olayer.balance_loss(counts, p, wl.alpha)
+    t_route = time.perf_counter() - t0
+
+    geom = W.stga_shape(wl)
+    scale = 1.0 / math.sqrt(wl.hd)
+    t_attn = 0.0
+    for h in heads:
+        qh, kh, vh = (W.bf16_bits_to_f64(inputs[n][:, h:h + 1, :]) for n in ("q", "k", "v"))
+        t0 = time.perf_counter()
+        om = oatt.moga(qh, kh, vh, g, p_g, wl.M, scale)
+        ow = oatt.grouped(qh, kh, vh, ostga.window_groups(geom), scale)
+        of = oatt.grouped(qh, kh, vh, ostga.frame_groups(geom), scale)
+        olayer.mean3(om, ow, of)
+        t_attn += time.perf_counter() - t0
+    t_layer = t_route + t_attn * (wl.H / len(heads))
+    return wl.N / t_layer, dict(t_route_s=t_route, t_attn_s=t_attn, heads=len(heads))
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = WORKLOAD
+    inputs = make_inputs(wl)
+    for i in range(args.warmup):
+        oracle_sample(wl, inputs, heads=(i % wl.H,))
+    t0 = time.perf_counter()
+    vals = [oracle_sample(wl, inputs, heads=(s % wl.H,))[0] for s in range(args.steps)]
+    el = time.perf_counter() - t0
+    value = float(statistics.median(vals))
+    sample = ("fp64 oracle per step: route+permute+loss over all %d tokens, attention (MoGA+window+frame+mean) "
+              "over all tokens for 1 of %d heads, extrapolated to all heads" % (wl.N, wl.H))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * el / max(args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(wl),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(wl):
+    return {"workload": wl.name, "tokens": wl.N, "frames": wl.T, "grid": [wl.h, wl.w], "d": wl.d,
+            "heads": wl.H, "head_dim": wl.hd, "M": wl.M, "shots": list(wl.shots), "tg_max": wl.tg_max,
+            "window": [wl.win_h, wl.win_w], "aug_frames": wl.aug, "sequences_per_gpu": 1,
+            "l2": "flushed between timed steps (256 MiB write)", "parallelism": "independent sequences per GPU"}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    import sparse_attention_long_moga_b200 as moga
+    wl = WORKLOAD
+    inp = make_inputs(wl)
+    geom = W.stga_shape(wl)
+
+    def to_dev(a):
+        t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+        return t.to(dev).view(torch.bfloat16) if a.dtype == np.uint16 else t.to(dev)
+
+    x, w_r, q, k, v = (to_dev(inp[n]) for n in ("x", "w_r", "q", "k", "v"))
+    N, M, H, hd = wl.N, wl.M, wl.H, wl.hd
+    L = moga._lib.lib()
+    stream = torch.cuda.current_stream()
+    sp = moga._stream()
+    P = moga._ptr
+
+    # persistent buffers: the step allocates nothing
+    g = torch.empty(N, dtype=torch.int32, device=dev)
+    gate = torch.empty(N, dtype=torch.float32, device=dev)
+    rws = torch.empty(max(L.moga_route_ws_bytes(N, M), 16), dtype=torch.uint8, device=dev)
+    pws = torch.empty(max(L.moga_permute_ws_bytes(N, M), 16), dtype=torch.uint8, device=dev)
+    perm = torch.empty(N, dtype=torch.int32, device=dev)
+    cu = torch.empty(M + 1, dtype=torch.int32, device=dev)
+    counts = torch.empty(M, dtype=torch.int32, device=dev)
+    mx = torch.empty(1, dtype=torch.int32, device=dev)
+    o_acc = torch.empty((N, H, hd), dtype=torch.float32, device=dev)
+    out = torch.empty((N, H, hd), dtype=torch.bfloat16, device=dev)
+    loss = torch.empty(1, dtype=torch.float64, device=dev)
+    gs, keep = moga.geom_struct(geom)
+    scale = 1.0 / math.sqrt(hd)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ev_moga = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+
+    def step(xd, qd, kd, vd, time_moga=False):
+        c = moga.check
+        c(L.moga_route(P(xd), P(w_r), moga.MOGA_BF16, None, N, wl.d, M, P(g), P(gate), P(rws), rws.numel(), sp),
+          "route")
+        c(L.moga_permute(P(g), N, M, P(perm), P(cu), P(counts), P(mx), P(pws), pws.numel(), sp), "permute")
+        if time_moga:
+            ev_moga[0].record(stream)
+        c(L.moga_group_attn(P(qd), P(kd), P(vd), N, H, hd, P(perm), P(cu), M, P(gate), scale, P(o_acc), sp), "moga")
+        if time_moga:
+            ev_moga[1].record(stream)
+        c(L.stga_attn(P(qd), P(kd), P(vd), H, hd, moga.ctypes.byref(gs), scale, P(o_acc), sp), "stga")
+        c(L.visual_attn_mean(P(o_acc), o_acc.numel(), P(out), sp), "mean")
+        c(L.moga_balance_loss(P(counts), P(rws), N, M, wl.alpha, P(loss), sp), "loss")
+
+    launches_per_step = 1 + 3 + 1 + 2 + 1 + 1 + (1 if (N * H * hd) % 8 else 0)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(x, q, k, v)
+    moga.device_status()
+
+    # ---- device-timed region: K steps, L2 flushed between steps
+    sampler = ClockSampler(local)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    moga_ms = []
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        step(x, q, k, v, time_moga=True)
+        evs[i][1].record(stream)
+        ev_moga[1].synchronize()
+        moga_ms.append(ev_moga[0].elapsed_time(ev_moga[1]))
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    moga.device_status()
+    dev_ms = sum(a.elapsed_time(b) for a, b in evs)
+    t = torch.tensor([dev_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.barrier()
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    job_ms = float(t.item())
+    value = world * N * args.steps / (job_ms / 1000.0)
+
+    # ---- end to end through the public API: pinned host inputs in, result out
+    hx, hq, hk, hv = (torch.from_numpy(inp[n].view(np.int16)).pin_memory() for n in ("x", "q", "k", "v"))
+    xd, qd, kd, vd = (torch.empty_like(a, device=dev) for a in (hx, hq, hk, hv))
+    hout = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    hloss = torch.empty(1, dtype=torch.float64).pin_memory()
+    h2d = sum(a.numel() * a.element_size() for a in (hx, hq, hk, hv))
+    d2h = hout.numel() * 2 + 8
+    e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        e_evs[i][0].record(stream)
+        for dst, src in ((xd, hx), (qd, hq), (kd, hk), (vd, hv)):
+            dst.copy_(src, non_blocking=True)
+        step(xd.view(torch.bfloat16), qd.view(torch.bfloat16), kd.view(torch.bfloat16), vd.view(torch.bfloat16))
+        hout.copy_(out, non_blocking=True)
+        hloss.copy_(loss, non_blocking=True)
+        e_evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e_evs)
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = world * N * args.steps / (float(te.item()) / 1000.0)
+
+    counts_h = counts.cpu().numpy()
+    fl_moga = moga_flops(counts_h, H, hd)
+    fl_stga = stga_flops(wl)
+    pk, pk_kind = peaks()
+    moga_avg_s = statistics.mean(moga_ms) / 1000.0
+    achieved = fl_moga / moga_avg_s / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": job_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded counter-based generator; no dataset)",
+        "config": config_dict(wl),
+        "roofline": {"bound": "tensor", "kernel": "group_attn_kernel<128> (MoGA groups)", "achieved": achieved,
+                     "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+                     "peak_kind": "%s burst dense bf16" % pk_kind, "traffic": None,
+                     "flops_per_launch": fl_moga, "launch_ms": moga_avg_s * 1e3},
+        "layer_tflops": (fl_moga + fl_stga) / (job_ms / args.steps / 1000.0) / 1e12,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu_val, det = oracle_sample(wl, inp, heads=(0, 1))
+        line["cpu_baseline"] = {"value": cpu_val, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+                                "sample": "fp64 oracle: route+permute+loss over all %d tokens, attention+mean over "
+                                          "all tokens for 2 of %d heads, extrapolated to all heads (%.1f s route, "
+                                          "%.1f s attention)" % (N, H, det["t_route_s"], det["t_attn_s"])}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    del keep
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
