@@ -102,6 +102,26 @@ moga_status moga_permute(const int32_t* group_id, int64_t N, int32_t M,
                          int32_t* perm, int32_t* cu_seqlens, int32_t* counts, int32_t* max_seqlen,
                          void* ws, size_t ws_bytes, void* stream);
 
+/* The same stable permute without a caller workspace.  The paper has no
+ * counterpart to this call; it exists for callers that cannot allocate device
+ * memory when they run the layer: code running inside another runtime's
+ * plugin or callback whose device memory that runtime owns, programs that
+ * plan a fixed device-memory budget up front and forbid cudaMalloc while
+ * serving (it can also stall the device), and C callers with no allocator at
+ * hand.  Scratch comes from a 512 KiB array the library keeps on each GPU
+ * that loads it, for the life of the process.
+ *   - N must be <= 4,194,304 (larger N returns MOGA_ERR_WORKSPACE, nothing
+ *     is launched); M in [1, 32].  Outputs as for moga_permute.
+ *   - All calls on one GPU share that array.  Calls whose kernels overlap on
+ *     the GPU (other streams or host threads) race on it: serialise them.
+ *     Nothing in it needs to start at zero; each call writes what it reads.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Allocates nothing and calls no allocating routine. */
+moga_status moga_permute_noalloc(const int32_t* group_id, int64_t N, int32_t M,
+                                 int32_t* perm, int32_t* cu_seqlens, int32_t* counts,
+                                 int32_t* max_seqlen, void* stream);
+
 /* -------------------------------------------------------- group attention --
  * MoGA attention (note, key designs 1-2): for every group i and head h,
  * full non-causal softmax attention among the tokens perm[cu[i] .. cu[i+1]),

@@ -3,5 +3,6 @@
 #include "api_common.cu"
 #include "route.cu"
 #include "permute.cu"
+#include "permute_noalloc.cu"
 #include "mean_loss.cu"
 #include "attention.cu"
