@@ -250,6 +250,7 @@ def run_ours(args):
     o_acc = torch.empty((N, H, hd), dtype=torch.float32, device=dev)
     out = torch.empty((N, H, hd), dtype=torch.bfloat16, device=dev)
     loss = torch.empty(1, dtype=torch.float64, device=dev)
+    aws = torch.empty(L.moga_attn_ws_bytes(N, H, hd), dtype=torch.uint8, device=dev)
     gs, keep = moga.geom_struct(geom)
     scale = 1.0 / math.sqrt(hd)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -262,14 +263,17 @@ def run_ours(args):
         c(L.moga_permute(P(g), N, M, P(perm), P(cu), P(counts), P(mx), P(pws), pws.numel(), sp), "permute")
         if time_moga:
             ev_moga[0].record(stream)
-        c(L.moga_group_attn(P(qd), P(kd), P(vd), N, H, hd, P(perm), P(cu), M, P(gate), scale, P(o_acc), sp), "moga")
+        c(L.moga_group_attn(P(qd), P(kd), P(vd), N, H, hd, P(perm), P(cu), M, P(gate), scale, P(o_acc), P(aws), aws.numel(), sp),
+          "moga")
         if time_moga:
             ev_moga[1].record(stream)
-        c(L.stga_attn(P(qd), P(kd), P(vd), H, hd, moga.ctypes.byref(gs), scale, P(o_acc), sp), "stga")
+        c(L.stga_attn(P(qd), P(kd), P(vd), H, hd, moga.ctypes.byref(gs), scale, P(o_acc), P(aws), aws.numel(),
+                        sp), "stga")
         c(L.visual_attn_mean(P(o_acc), o_acc.numel(), P(out), sp), "mean")
         c(L.moga_balance_loss(P(counts), P(rws), N, M, wl.alpha, P(loss), sp), "loss")
 
-    launches_per_step = 1 + 3 + 1 + 2 + 1 + 1 + (1 if (N * H * hd) % 8 else 0)
+    # route 1, permute 3, MoGA gather + attention 2, STGA gather + window + frame 3, mean 1 (+tail), loss 1
+    launches_per_step = 1 + 3 + 2 + 3 + 1 + 1 + (1 if (N * H * hd) % 8 else 0)
 
     for _ in range(args.warmup):
         flush.zero_()

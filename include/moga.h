@@ -122,6 +122,14 @@ moga_status moga_permute_noalloc(const int32_t* group_id, int64_t N, int32_t M,
                                  int32_t* perm, int32_t* cu_seqlens, int32_t* counts,
                                  int32_t* max_seqlen, void* stream);
 
+/* ------------------------------------------------------ attention scratch --
+ * Both attention calls first copy Q, K and V into segment order (rows of a
+ * group contiguous) so that the attention kernel streams whole tiles; they
+ * need a caller workspace of at least moga_attn_ws_bytes(N, H, hd) bytes
+ * (3 * N * H * hd * 2).  One workspace can serve both calls on one stream.
+ * Returns 0 for arguments the calls would reject. */
+size_t moga_attn_ws_bytes(int64_t N, int32_t H, int32_t hd);
+
 /* -------------------------------------------------------- group attention --
  * MoGA attention (note, key designs 1-2): for every group i and head h,
  * full non-causal softmax attention among the tokens perm[cu[i] .. cu[i+1]),
@@ -131,12 +139,13 @@ moga_status moga_permute_noalloc(const int32_t* group_id, int64_t N, int32_t M,
  * o_acc:    [N][H][hd] fp32, OVERWRITTEN for every token (empty groups are
  *           skipped; tokens are covered because perm is a permutation)
  * softmax_scale: usually 1/sqrt(hd).
+ * ws:       attention workspace (see moga_attn_ws_bytes), 16-byte aligned.
  */
 moga_status moga_group_attn(const void* q, const void* k, const void* v,
                             int64_t N, int32_t H, int32_t hd,
                             const int32_t* perm, const int32_t* cu_seqlens, int32_t M,
                             const float* gate_prob, float softmax_scale,
-                            float* o_acc, void* stream);
+                            float* o_acc, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------- STGA --
  * Static spatial-temporal group attention plus per-frame attention (note,
@@ -145,10 +154,11 @@ moga_status moga_group_attn(const void* q, const void* k, const void* v,
  *             + SA(q_t, K/V of its latent frame).
  * q, k, v: [N][H][hd] bf16 with N = T*h*w;  o_acc: [N][H][hd] fp32, ADDED TO.
  * geom: HOST pointer, read during the call only.
+ * ws:   attention workspace (see moga_attn_ws_bytes), 16-byte aligned.
  */
 moga_status stga_attn(const void* q, const void* k, const void* v, int32_t H, int32_t hd,
                       const moga_stga_geom* geom, float softmax_scale,
-                      float* o_acc, void* stream);
+                      float* o_acc, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------- mean --
  * Three-way mean (note, flowchart "多组输出取均值" and key design 4):

@@ -23,7 +23,7 @@ import torch
 from ._lib import MOGA_BF16, MOGA_F32, MogaError, StgaGeom, check, lib  # noqa: F401
 
 __all__ = ["moga_route", "moga_permute", "moga_group_attn", "stga_attn", "visual_attn_mean",
-           "moga_balance_loss", "visual_attention_forward", "device_status", "MogaError", "geom_struct"]
+           "moga_balance_loss", "visual_attention_forward", "attn_workspace", "device_status", "MogaError", "geom_struct"]
 
 
 def _ptr(t):
@@ -93,8 +93,17 @@ def _check_qkv(q, k, v):
     return q.shape
 
 
+def attn_workspace(q: torch.Tensor) -> torch.Tensor:
+    """Scratch for the attention calls (Q, K, V copied into segment order)."""
+    N, H, hd = q.shape
+    n = lib().moga_attn_ws_bytes(N, H, hd)
+    if n == 0:
+        raise ValueError("unsupported attention shape %s" % (tuple(q.shape),))
+    return torch.empty(n, dtype=torch.uint8, device=q.device)
+
+
 def moga_group_attn(q, k, v, perm, cu_seqlens, gate_prob, M: int, softmax_scale: float | None = None,
-                    o_acc: torch.Tensor | None = None):
+                    o_acc: torch.Tensor | None = None, ws: torch.Tensor | None = None):
     """o_acc[perm[j]] = gate * softmax(q k^T * scale) v inside each group (written, fp32)."""
     N, H, hd = _check_qkv(q, k, v)
     _need(perm, torch.int32, "perm", 1)
@@ -104,8 +113,10 @@ def moga_group_attn(q, k, v, perm, cu_seqlens, gate_prob, M: int, softmax_scale:
         o_acc = torch.empty((N, H, hd), dtype=torch.float32, device=q.device)
     _need(o_acc, torch.float32, "o_acc", 3)
     scale = 1.0 / math.sqrt(hd) if softmax_scale is None else softmax_scale
+    ws = attn_workspace(q) if ws is None else ws
     check(lib().moga_group_attn(_ptr(q), _ptr(k), _ptr(v), N, H, hd, _ptr(perm), _ptr(cu_seqlens), M,
-                                _ptr(gate_prob), scale, _ptr(o_acc), _stream()), "moga_group_attn")
+                                _ptr(gate_prob), scale, _ptr(o_acc), _ptr(ws), ws.numel(), _stream()),
+          "moga_group_attn")
     return o_acc
 
 
@@ -117,7 +128,8 @@ def geom_struct(geom: dict):
     return s, shots
 
 
-def stga_attn(q, k, v, geom: dict, softmax_scale: float | None = None, o_acc: torch.Tensor | None = None):
+def stga_attn(q, k, v, geom: dict, softmax_scale: float | None = None, o_acc: torch.Tensor | None = None,
+              ws: torch.Tensor | None = None):
     """o_acc += window-group attention + per-frame attention (fp32)."""
     N, H, hd = _check_qkv(q, k, v)
     if o_acc is None:
@@ -125,8 +137,9 @@ def stga_attn(q, k, v, geom: dict, softmax_scale: float | None = None, o_acc: to
     _need(o_acc, torch.float32, "o_acc", 3)
     scale = 1.0 / math.sqrt(hd) if softmax_scale is None else softmax_scale
     s, keep = geom_struct(geom)
-    check(lib().stga_attn(_ptr(q), _ptr(k), _ptr(v), H, hd, ctypes.byref(s), scale, _ptr(o_acc), _stream()),
-          "stga_attn")
+    ws = attn_workspace(q) if ws is None else ws
+    check(lib().stga_attn(_ptr(q), _ptr(k), _ptr(v), H, hd, ctypes.byref(s), scale, _ptr(o_acc), _ptr(ws),
+                          ws.numel(), _stream()), "stga_attn")
     del keep
     return o_acc
 
@@ -161,8 +174,9 @@ def visual_attention_forward(x, w_r, bias, q, k, v, M: int, geom: dict, alpha: f
     """The whole layer: returns dict(out bf16 [N,H,hd], loss fp64 [1], g, gate, perm, cu_seqlens, counts)."""
     g, gate, ws = moga_route(x, w_r, bias)
     perm, cu, counts, mx = moga_permute(g, M)
-    o = moga_group_attn(q, k, v, perm, cu, gate, M, softmax_scale)
-    stga_attn(q, k, v, geom, softmax_scale, o_acc=o)
+    ws_attn = attn_workspace(q)
+    o = moga_group_attn(q, k, v, perm, cu, gate, M, softmax_scale, ws=ws_attn)
+    stga_attn(q, k, v, geom, softmax_scale, o_acc=o, ws=ws_attn)
     out = visual_attn_mean(o)
     loss = moga_balance_loss(counts, ws, x.shape[0], M, alpha)
     return dict(out=out, loss=loss, g=g, gate=gate, perm=perm, cu_seqlens=cu, counts=counts, max_seqlen=mx)

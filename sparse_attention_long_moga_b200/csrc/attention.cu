@@ -8,18 +8,25 @@
 // written back at the token's own row (no repermute pass).  The static
 // groups add their outputs into the same fp32 accumulator.
 //
-// Structure of one CTA (one 128-row query tile of one group and one head):
-//   warps 0-3  softmax + epilogue: thread = query row = TMEM lane
-//   warp  4    producer: TMA tile::gather4 of Q/K/V rows, rows chosen by an
-//              index map (perm for MoGA, window arithmetic for STGA,
-//              identity for frames); 128B-swizzled tiles
-//   warp  5    TMEM allocator; lane 0 issues tcgen05.mma
-// TMEM columns: S double buffer [0,128) and [128,256), O at [256, 256+hd).
-// Pipeline per KV tile j: S_j = Q K_j^T (MMA) -> row max, exp2, P_j -> bf16
-// into shared memory (softmax warps) -> O += P_j V_j (MMA).  The MMA of
-// S_{j+1} overlaps the softmax of tile j.  The running max is only moved
-// (and O rescaled) when it grows by more than 2^8, which keeps the result
-// exact while skipping most rescales.
+// Two kernels per branch:
+//   gather3_kernel   HBM-bound row copy of Q, K, V into segment order (rows
+//                    picked through perm for MoGA, through the window map for
+//                    the static windows), so that every group is a contiguous
+//                    row range.  Frames are contiguous already and skip it.
+//   attn_kernel      one CTA per (group, head, pair of 128-row query tiles):
+//     warps 0-3 / 4-7  softmax + epilogue of query tile 0 / 1
+//                      (thread = query row = TMEM lane)
+//     warp 8           producer: 3-D tiled TMA loads (128B swizzle) of the
+//                      two Q tiles and a 2-stage ring of K and V tiles
+//     warp 9           TMEM allocator; lane 0 issues tcgen05.mma
+//   TMEM columns: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+//   The softmax writes P as bf16 pairs over the first 64 columns of its S
+//   and the P.V product reads it from there (A operand in tensor memory).
+//   Issue order per KV tile j:  PV0_j, S0_{j+1}, PV1_j, S1_{j+1}, so the
+//   softmax of one tile runs while the tensor core serves the other.
+//   The running row max only moves (and O is rescaled) when it grows by
+//   more than 2^8; the final 1/l uses the same reference, so the result is
+//   exact.
 // Every wait is bounded; on a timeout the CTA records MOGA_ERR_TIMEOUT,
 // drains what it has in flight, frees TMEM and exits.
 #include <cuda.h>
@@ -34,9 +41,9 @@
 namespace moga {
 namespace attn {
 
-constexpr int BM = 128;        // query rows per tile
+constexpr int BM = 128;        // query rows per tile (two tiles per CTA)
 constexpr int BN = 128;        // key/value rows per tile
-constexpr int kThreads = 192;  // 6 warps
+constexpr int kThreads = 320;  // 10 warps
 constexpr int kMaxTG = 256;    // temporal groups per launch
 constexpr uint32_t kTmemCols = 512;
 constexpr int kHalfBytes = BM * 128;   // one 64-column half of a 128-row tile (16 KB)
@@ -60,7 +67,7 @@ struct Params {
   // STGA geometry
   int T, h, w, win_h, win_w, n_wx, n_win, whw, hw;
   int n_tg;
-  int tg_tiles[kMaxTG + 1];   // prefix of tiles over temporal groups
+  int tg_tiles[kMaxTG + 1];   // prefix of CTAs over temporal groups
   TGroup tg[kMaxTG];
   long long timeout_cycles;
   int debug_flags;            // bit 0: producer skips the Q load (timeout test)
@@ -111,7 +118,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
-// Bounded wait that ignores the abort flag (draining in-flight copies).
+// Bounded wait that ignores the abort flag (draining in-flight work).
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, long long timeout) {
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
@@ -122,12 +129,13 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, long l
   }
 }
 
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int col, int r0, int r1, int r2,
-                                            int r3, uint32_t bar) {
+// 3-D tiled TMA load: box {64 columns, 1 head, 128 rows}.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int col, int head, int row,
+                                            uint32_t bar) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(head), "r"(row), "r"(bar)
       : "memory");
 }
 
@@ -138,12 +146,23 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accumulate) {
+// D (tmem) (+)= A (smem desc) x B (smem desc)
+__device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
   asm volatile(
       "{ .reg .pred p; setp.ne.b32 p, %4, 0;"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D (tmem) (+)= A (tmem) x B (smem desc)
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0;"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -180,6 +199,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
       : "memory");
 }
 
+// 32 lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -187,6 +216,11 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
@@ -208,14 +242,10 @@ __host__ __device__ constexpr uint32_t instr_desc(int n, bool b_mn_major) {
 
 // ------------------------------------------------------------------ index maps
 
-struct Tile {
-  int head, q_begin, q_end, kv_begin, kv_end;
-  int valid;  // 0: this CTA has no work
-};
-
-__device__ __forceinline__ int token_of(const Params& p, int idx) {
-  if (p.mode == MODE_MOGA) return __ldg(p.perm + idx);
-  if (p.mode == MODE_FRAME) return idx;
+// Token at position idx of the window-major order (window, frame, position
+// inside the window), in which a temporal group's keys/values -- including
+// the frames borrowed from the neighbouring shots -- are one contiguous range.
+__device__ __forceinline__ int window_token(const Params& p, int idx) {
   const int local = idx % p.whw;
   const int wf = idx / p.whw;
   const int frame = wf % p.T;
@@ -226,12 +256,24 @@ __device__ __forceinline__ int token_of(const Params& p, int idx) {
   return frame * p.hw + row * p.w + col;
 }
 
-// Decode blockIdx into a tile (thread 0 only; result shared via smem).
+__device__ __forceinline__ int token_of(const Params& p, int idx) {
+  if (p.mode == MODE_MOGA) return __ldg(p.perm + idx);
+  if (p.mode == MODE_FRAME) return idx;
+  return window_token(p, idx);
+}
+
+struct Tile {
+  int head, q_begin, q_end, kv_begin, kv_end;
+  int valid;  // 0: this CTA has no work
+};
+
+// Decode blockIdx into a tile pair (thread 0 only; shared through smem).
 __device__ void decode_tile(const Params& p, int L, Tile& t) {
   t.valid = 0;
+  constexpr int kPair = 2 * BM;
   if (p.mode == MODE_MOGA) {
-    // largest groups first, then head, then query tile (K/V of one group and
-    // head are reused by consecutive CTAs through L2)
+    // largest groups first, then head, then query-tile pair (K/V of one group
+    // and head are reused by consecutive CTAs through L2)
     int size[32], order[32];
     for (int i = 0; i < p.M; ++i) {
       size[i] = __ldg(p.cu + i + 1) - __ldg(p.cu + i);
@@ -249,14 +291,14 @@ __device__ void decode_tile(const Params& p, int L, Tile& t) {
     int rem = L;
     for (int k = 0; k < p.M; ++k) {
       const int g = order[k];
-      const int qt = ceil_div(size[g], BM);
-      const int n = qt * p.H;
+      const int qp = ceil_div(size[g], kPair);
+      const int n = qp * p.H;
       if (rem < n) {
         const int start = __ldg(p.cu + g);
-        t.head = rem / qt;
-        const int qi = rem - t.head * qt;
-        t.q_begin = start + qi * BM;
-        t.q_end = min(start + size[g], t.q_begin + BM);
+        t.head = rem / qp;
+        const int qi = rem - t.head * qp;
+        t.q_begin = start + qi * kPair;
+        t.q_end = min(start + size[g], t.q_begin + kPair);
         t.kv_begin = start;
         t.kv_end = start + size[g];
         t.valid = 1;
@@ -267,38 +309,62 @@ __device__ void decode_tile(const Params& p, int L, Tile& t) {
     return;
   }
   if (p.mode == MODE_FRAME) {
-    const int qt = ceil_div(p.hw, BM);
-    const int total = p.T * p.H * qt;
+    const int qp = ceil_div(p.hw, kPair);
+    const int total = p.T * p.H * qp;
     if (L >= total) return;
-    const int frame = L / (p.H * qt);
-    const int rem = L - frame * p.H * qt;
-    t.head = rem / qt;
-    const int qi = rem - t.head * qt;
+    const int frame = L / (p.H * qp);
+    const int rem = L - frame * p.H * qp;
+    t.head = rem / qp;
+    const int qi = rem - t.head * qp;
     t.kv_begin = frame * p.hw;
     t.kv_end = t.kv_begin + p.hw;
-    t.q_begin = t.kv_begin + qi * BM;
-    t.q_end = min(t.kv_end, t.q_begin + BM);
+    t.q_begin = t.kv_begin + qi * kPair;
+    t.q_end = min(t.kv_end, t.q_begin + kPair);
     t.valid = 1;
     return;
   }
-  // window groups: temporal group, window, head, query tile
+  // window groups: temporal group, window, head, query-tile pair
   if (L >= p.tg_tiles[p.n_tg]) return;
   int g = 0;
   while (p.tg_tiles[g + 1] <= L) ++g;
   const TGroup tg = p.tg[g];
   const int qlen = (tg.t1 - tg.t0) * p.whw;
-  const int qt = ceil_div(qlen, BM);
+  const int qp = ceil_div(qlen, kPair);
   const int rem = L - p.tg_tiles[g];
-  const int win = rem / (p.H * qt);
-  const int rem2 = rem - win * p.H * qt;
-  t.head = rem2 / qt;
-  const int qi = rem2 - t.head * qt;
+  const int win = rem / (p.H * qp);
+  const int rem2 = rem - win * p.H * qp;
+  t.head = rem2 / qp;
+  const int qi = rem2 - t.head * qp;
   const int base = win * p.T;
-  t.q_begin = (base + tg.t0) * p.whw + qi * BM;
-  t.q_end = min((base + tg.t1) * p.whw, t.q_begin + BM);
+  t.q_begin = (base + tg.t0) * p.whw + qi * kPair;
+  t.q_end = min((base + tg.t1) * p.whw, t.q_begin + kPair);
   t.kv_begin = (base + tg.t0 - tg.a_prev) * p.whw;
   t.kv_end = (base + tg.t1 + tg.a_next) * p.whw;
   t.valid = 1;
+}
+
+// ------------------------------------------------------------------ gather
+
+// dst[j] = src[map(j)] for the rows of Q, K and V ([N][H*hd] bf16, rows of
+// `row_u4` 16-byte vectors); one warp per destination row.
+template <int MODE>
+__global__ void __launch_bounds__(256)
+gather3_kernel(const __grid_constant__ Params p, const uint4* __restrict__ q, const uint4* __restrict__ k,
+               const uint4* __restrict__ v, uint4* __restrict__ qd, uint4* __restrict__ kd, uint4* __restrict__ vd,
+               int row_u4) {
+  const int j = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (j >= p.N) return;
+  const int lane = threadIdx.x & 31;
+  const int src = MODE == MODE_MOGA ? __ldg(p.perm + j) : window_token(p, j);
+  const size_t so = (size_t)src * row_u4, dofs = (size_t)j * row_u4;
+  for (int c = lane; c < row_u4; c += 32) {
+    const uint4 a = __ldg(q + so + c);
+    const uint4 b = __ldg(k + so + c);
+    const uint4 e = __ldg(v + so + c);
+    qd[dofs + c] = a;
+    kd[dofs + c] = b;
+    vd[dofs + c] = e;
+  }
 }
 
 // ------------------------------------------------------------------ shared memory
@@ -306,17 +372,16 @@ __device__ void decode_tile(const Params& p, int L, Tile& t) {
 template <int HD>
 struct SmemLayout {
   static constexpr int kHalves = HD / 64;
-  static constexpr int kTileBytes = kHalves * kHalfBytes;  // one Q/K/V tile
-  static constexpr int kQ = 0;
-  static constexpr int kK0 = kQ + kTileBytes;
-  static constexpr int kV0 = kK0 + 2 * kTileBytes;
-  static constexpr int kP = kV0 + 2 * kTileBytes;
-  static constexpr int kBar = kP + 2 * kHalfBytes;
+  static constexpr int kTileBytes = kHalves * kHalfBytes;  // one 128-row Q/K/V tile
+  static constexpr int kQ = 0;                              // two Q tiles
+  static constexpr int kK0 = kQ + 2 * kTileBytes;           // two K stages
+  static constexpr int kV0 = kK0 + 2 * kTileBytes;          // two V stages
+  static constexpr int kBar = kV0 + 2 * kTileBytes;
   static constexpr int kNumBars = 16;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kEnd = kMisc + 64;
-  // 1 KB slack to align the dynamic base to 1024 bytes; HD = 64 is padded so
-  // two CTAs never share an SM (each allocates all 512 TMEM columns)
+  // 1 KB slack to align the dynamic base to 1024 bytes; the hd = 64 layout is
+  // padded so that two CTAs never share an SM (each holds all 512 TMEM columns)
   static constexpr int kBytes = (HD == 64 ? 120 * 1024 : kEnd) + 1024;
 };
 
@@ -326,19 +391,18 @@ enum Bar : int {
   B_FULL_V = 3,   // +stage
   B_EMPTY_K = 5,  // +stage
   B_EMPTY_V = 7,  // +stage
-  B_S_FULL = 9,   // +buffer
-  B_S_FREE = 11,  // +buffer
-  B_P_FULL = 13,
-  B_O_DONE = 14,
-  B_MMA_END = 15
+  B_S_FULL = 9,   // +query tile
+  B_P_FULL = 11,  // +query tile
+  B_O_FULL = 13,
+  B_MMA_END = 14
 };
 
 // ------------------------------------------------------------------ the kernel
 
 template <int HD>
-__global__ void __launch_bounds__(kThreads, 1)
-group_attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tm_q,
-                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
+__global__ void __launch_bounds__(kThreads)
+attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tm_q,
+            const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
   using S = SmemLayout<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -363,18 +427,18 @@ group_attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUte
       mbar_init(bar(B_EMPTY_K + s), 1);
       mbar_init(bar(B_EMPTY_V + s), 1);
       mbar_init(bar(B_S_FULL + s), 1);
-      mbar_init(bar(B_S_FREE + s), BM);
+      mbar_init(bar(B_P_FULL + s), BM);
     }
-    mbar_init(bar(B_P_FULL), BM);
-    mbar_init(bar(B_O_DONE), 1);
+    mbar_init(bar(B_O_FULL), 1);
     mbar_init(bar(B_MMA_END), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
   const Tile t = *tile_sh;
   if (!t.valid) return;   // uniform across the CTA
+  const bool has_q1 = t.q_begin + BM < t.q_end;
 
-  if (warp == 5) {
+  if (warp == 9) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(kTmemCols)
                  : "memory");
@@ -384,128 +448,134 @@ group_attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUte
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_o = tmem + 256;
   const long long timeout = p.timeout_cycles;
   const int n_kv = ceil_div(t.kv_end - t.kv_begin, BN);
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ---------------------------------------------------------------- producer
-    // lane l gathers rows 4l .. 4l+3 of every tile
-    auto rows_of = [&](int begin, int end, int* r) {
+    if (lane == 0) {
+      const bool skip_q = (p.debug_flags & 1) != 0;
+      int issued_k[2] = {-1, -1}, issued_v[2] = {-1, -1};
+      if (!skip_q) {
+        mbar_arrive_expect_tx(bar(B_FULL_Q), (has_q1 ? 2 : 1) * S::kTileBytes);
+        for (int qt = 0; qt < (has_q1 ? 2 : 1); ++qt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int idx = min(begin + 4 * lane + i, end - 1);
-        r[i] = token_of(p, idx) * p.H + t.head;
+          for (int hh = 0; hh < S::kHalves; ++hh)
+            tma_load_3d(sbase + S::kQ + qt * S::kTileBytes + hh * kHalfBytes, &tm_q, hh * 64, t.head,
+                        t.q_begin + qt * BM, bar(B_FULL_Q));
       }
-    };
-    auto issue_tile = [&](const CUtensorMap* map, uint32_t dst, const int* r, uint32_t b) {
+      for (int j = 0; j < n_kv; ++j) {
+        const int st = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        const int row = t.kv_begin + j * BN;
+        if (!mbar_wait(bar(B_EMPTY_K + st), ph ^ 1, abort_flag, timeout)) break;
+        mbar_arrive_expect_tx(bar(B_FULL_K + st), S::kTileBytes);
 #pragma unroll
-      for (int hh = 0; hh < S::kHalves; ++hh)
-        tma_gather4(dst + hh * kHalfBytes + lane * 512, map, hh * 64, r[0], r[1], r[2], r[3], b);
-    };
-    bool ok = true;
-    int issued_k[2] = {-1, -1}, issued_v[2] = {-1, -1};
-    const bool skip_q = (p.debug_flags & 1) != 0;
-    if (!skip_q) {
-      int r[4];
-      rows_of(t.q_begin, t.q_end, r);
-      if (lane == 0) mbar_arrive_expect_tx(bar(B_FULL_Q), S::kTileBytes);
-      __syncwarp();
-      issue_tile(&tm_q, sbase + S::kQ, r, bar(B_FULL_Q));
+        for (int hh = 0; hh < S::kHalves; ++hh)
+          tma_load_3d(sbase + S::kK0 + st * S::kTileBytes + hh * kHalfBytes, &tm_k, hh * 64, t.head, row,
+                      bar(B_FULL_K + st));
+        issued_k[st] = j;
+        if (!mbar_wait(bar(B_EMPTY_V + st), ph ^ 1, abort_flag, timeout)) break;
+        mbar_arrive_expect_tx(bar(B_FULL_V + st), S::kTileBytes);
+#pragma unroll
+        for (int hh = 0; hh < S::kHalves; ++hh)
+          tma_load_3d(sbase + S::kV0 + st * S::kTileBytes + hh * kHalfBytes, &tm_v, hh * 64, t.head, row,
+                      bar(B_FULL_V + st));
+        issued_v[st] = j;
+      }
+      // let every copy started here land before the CTA can exit
+      if (!skip_q) mbar_drain(bar(B_FULL_Q), 0, timeout);
+      for (int st = 0; st < 2; ++st) {
+        if (issued_k[st] >= 0) mbar_drain(bar(B_FULL_K + st), (issued_k[st] >> 1) & 1, timeout);
+        if (issued_v[st] >= 0) mbar_drain(bar(B_FULL_V + st), (issued_v[st] >> 1) & 1, timeout);
+      }
     }
-    for (int j = 0; j < n_kv && ok; ++j) {
-      const int st = j & 1;
-      const uint32_t ph = (j >> 1) & 1;
-      int r[4];
-      rows_of(t.kv_begin + j * BN, t.kv_end, r);
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_EMPTY_K + st), ph ^ 1, abort_flag, timeout));
-      if (!ok) break;
-      if (lane == 0) mbar_arrive_expect_tx(bar(B_FULL_K + st), S::kTileBytes);
-      __syncwarp();
-      issue_tile(&tm_k, sbase + S::kK0 + st * S::kTileBytes, r, bar(B_FULL_K + st));
-      issued_k[st] = j;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_EMPTY_V + st), ph ^ 1, abort_flag, timeout));
-      if (!ok) break;
-      if (lane == 0) mbar_arrive_expect_tx(bar(B_FULL_V + st), S::kTileBytes);
-      __syncwarp();
-      issue_tile(&tm_v, sbase + S::kV0 + st * S::kTileBytes, r, bar(B_FULL_V + st));
-      issued_v[st] = j;
-    }
-    // let every copy this warp started land before the CTA can exit
-    if (!skip_q) mbar_drain(bar(B_FULL_Q), 0, timeout);
-    for (int st = 0; st < 2; ++st) {
-      if (issued_k[st] >= 0) mbar_drain(bar(B_FULL_K + st), (issued_k[st] >> 1) & 1, timeout);
-      if (issued_v[st] >= 0) mbar_drain(bar(B_FULL_V + st), (issued_v[st] >> 1) & 1, timeout);
-    }
-  } else if (warp == 5) {
+    __syncwarp();
+  } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = instr_desc(BN, false);
       constexpr uint32_t idesc_pv = instr_desc(HD, true);
-      bool ok = mbar_wait(bar(B_FULL_Q), 0, abort_flag, timeout);
-      auto issue_pv = [&](int i) -> bool {
-        const int st = i & 1;
-        const uint32_t ph = (i >> 1) & 1;
-        if (!mbar_wait(bar(B_FULL_V + st), ph, abort_flag, timeout)) return false;
-        if (!mbar_wait(bar(B_P_FULL), i & 1, abort_flag, timeout)) return false;
-        tc_fence_after();
-        const uint32_t pa = sbase + S::kP;
-        const uint32_t va = sbase + S::kV0 + st * S::kTileBytes;
-#pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks) {
-          const uint64_t ad = smem_desc(pa + (ks >> 2) * kHalfBytes + (ks & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc(va + ks * 16 * 128, kHalfBytes, 1024);
-          tc_mma(tmem_o, ad, bd, idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
-        }
-        tc_commit(bar(B_O_DONE));
-        tc_commit(bar(B_EMPTY_V + st));
-        return true;
-      };
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        ok = mbar_wait(bar(B_FULL_K + st), ph, abort_flag, timeout) &&
-             mbar_wait(bar(B_S_FREE + st), ph ^ 1, abort_flag, timeout);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t qa = sbase + S::kQ;
-        const uint32_t ka = sbase + S::kK0 + st * S::kTileBytes;
+      const uint32_t tmem_s[2] = {tmem, tmem + 128};
+      const uint32_t tmem_o[2] = {tmem + 256, tmem + 384};
+      const int nq = has_q1 ? 2 : 1;
+      auto issue_s = [&](int qt, int j) {
+        const uint32_t qa = sbase + S::kQ + qt * S::kTileBytes;
+        const uint32_t ka = sbase + S::kK0 + (j & 1) * S::kTileBytes;
 #pragma unroll
         for (int ks = 0; ks < HD / 16; ++ks) {
           const uint64_t ad = smem_desc(qa + (ks >> 2) * kHalfBytes + (ks & 3) * 32, 16, 1024);
           const uint64_t bd = smem_desc(ka + (ks >> 2) * kHalfBytes + (ks & 3) * 32, 16, 1024);
-          tc_mma(tmem + st * 128, ad, bd, idesc_qk, ks > 0 ? 1u : 0u);
+          tc_mma_ss(tmem_s[qt], ad, bd, idesc_qk, ks > 0 ? 1u : 0u);
         }
-        tc_commit(bar(B_S_FULL + st));
-        tc_commit(bar(B_EMPTY_K + st));
-        if (j > 0) ok = issue_pv(j - 1);
+        tc_commit(bar(B_S_FULL + qt));
+      };
+      auto issue_pv = [&](int qt, int j) {
+        const uint32_t va = sbase + S::kV0 + (j & 1) * S::kTileBytes;
+#pragma unroll
+        for (int ks = 0; ks < BN / 16; ++ks) {
+          const uint64_t bd = smem_desc(va + ks * 16 * 128, kHalfBytes, 1024);
+          tc_mma_ts(tmem_o[qt], tmem_s[qt] + ks * 8, bd, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(bar(B_FULL_Q), 0, abort_flag, timeout) &&
+                mbar_wait(bar(B_FULL_K + 0), 0, abort_flag, timeout);
+      if (ok) {
+        tc_fence_after();
+        for (int qt = 0; qt < nq; ++qt) issue_s(qt, 0);
+        tc_commit(bar(B_EMPTY_K + 0));
       }
-      if (ok) issue_pv(n_kv - 1);
-      // every MMA this thread issued has finished before TMEM is released
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int st = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        const bool more = j + 1 < n_kv;
+        ok = mbar_wait(bar(B_FULL_V + st), ph, abort_flag, timeout) &&
+             mbar_wait(bar(B_P_FULL + 0), j & 1, abort_flag, timeout);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        if (more) {
+          ok = mbar_wait(bar(B_FULL_K + ((j + 1) & 1)), ((j + 1) >> 1) & 1, abort_flag, timeout);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        if (has_q1) {
+          ok = mbar_wait(bar(B_P_FULL + 1), j & 1, abort_flag, timeout);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(1, j);
+        }
+        tc_commit(bar(B_EMPTY_V + st));
+        if (more) {
+          if (has_q1) issue_s(1, j + 1);
+          tc_commit(bar(B_EMPTY_K + ((j + 1) & 1)));
+        }
+      }
+      if (ok) tc_commit(bar(B_O_FULL));
+      // every MMA issued here has finished before TMEM is released
       tc_commit(bar(B_MMA_END));
       mbar_drain(bar(B_MMA_END), 0, timeout);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 4 || has_q1) {
     // ---------------------------------------------------------------- softmax
-    const int row = warp * 32 + lane;                    // TMEM lane == query row
-    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+    const int qt = warp >> 2;                            // query tile of this warpgroup
+    const int row = (warp & 3) * 32 + lane;              // TMEM lane == query row
+    const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t s_addr = tmem + lane_addr + qt * 128;
+    const uint32_t o_addr = tmem + lane_addr + 256 + qt * 128;
     const float sl = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    uint8_t* prow = smem + S::kP + row * 128;
     for (int j = 0; j < n_kv; ++j) {
-      const int sb = j & 1;
-      const uint32_t ph = (j >> 1) & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + sb), ph, abort_flag, timeout));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + qt), j & 1, abort_flag, timeout));
       if (!ok) break;
       tc_fence_after();
       float s[BN];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(tmem + lane_addr + sb * 128 + c * 32, s + c * 32);
+      for (int c = 0; c < BN / 32; ++c) tmem_ld32(s_addr + c * 32, s + c * 32);
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(B_S_FREE + sb));
       const int valid = t.kv_end - (t.kv_begin + j * BN);
       if (valid < BN) {
 #pragma unroll
@@ -516,57 +586,53 @@ group_attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUte
 #pragma unroll
       for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
       const float m_new = fmaxf(m_run, mx * sl);
-      if (j > 0) {
-        // PV_{j-1} has finished: P may be overwritten and O rescaled
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O_DONE), (j - 1) & 1, abort_flag, timeout));
-        if (!ok) break;
-        tc_fence_after();
+      if (j == 0) {
+        m_run = m_new;
+      } else {
+        // P.V of tile j-1 finished before S of tile j (issue order), so O may
+        // be rescaled here
         const bool need = m_new > m_run + 8.0f;
         if (__any_sync(0xffffffffu, need)) {
           const float f = need ? fast_exp2(m_run - m_new) : 1.0f;
 #pragma unroll 1
           for (int c = 0; c < HD / 32; ++c) {
             float o[32];
-            tmem_ld32(tmem_o + lane_addr + c * 32, o);
+            tmem_ld32(o_addr + c * 32, o);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] *= f;
-            tmem_st32(tmem_o + lane_addr + c * 32, o);
+            tmem_st32(o_addr + c * 32, o);
           }
-          tmem_wait_st();
           if (need) {
             l_run *= f;
             m_run = m_new;
           }
         }
-      } else {
-        m_run = m_new;
       }
+      const float neg_m = -m_run;
       float sum = 0.f;
 #pragma unroll
-      for (int c8 = 0; c8 < BN / 8; ++c8) {
-        uint32_t w[4];
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float a = fast_exp2(fmaf(s[c8 * 8 + 2 * i], sl, -m_run));
-          const float b = fast_exp2(fmaf(s[c8 * 8 + 2 * i + 1], sl, -m_run));
+        for (int i = 0; i < 16; ++i) {
+          const float a = fast_exp2(fmaf(s[c * 32 + 2 * i], sl, neg_m));
+          const float b = fast_exp2(fmaf(s[c * 32 + 2 * i + 1], sl, neg_m));
           sum += a + b;
-          __nv_bfloat162 pr = __floats2bfloat162_rn(a, b);
-          w[i] = *reinterpret_cast<uint32_t*>(&pr);
+          pk[i] = pack_bf16x2(a, b);
         }
-        const int half = c8 >> 3, chunk = c8 & 7;
-        const int off = half * kHalfBytes + ((chunk ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4*>(prow + off) = make_uint4(w[0], w[1], w[2], w[3]);
+        // P overwrites S columns [16c, 16c+16), whose scores were read above
+        tmem_st16(s_addr + c * 16, pk);
       }
       l_run += sum;
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(B_P_FULL));
+      mbar_arrive(bar(B_P_FULL + qt));
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O_DONE), (n_kv - 1) & 1, abort_flag, timeout));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O_FULL), 0, abort_flag, timeout));
     if (ok) {
       tc_fence_after();
-      const int q_idx = t.q_begin + row;
+      const int q_idx = t.q_begin + qt * BM + row;
       const bool live = q_idx < t.q_end;
       float scale = 0.f;
       float* dst = nullptr;
@@ -579,7 +645,7 @@ group_attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUte
 #pragma unroll 1
       for (int c = 0; c < HD / 32; ++c) {
         float o[32];
-        tmem_ld32(tmem_o + lane_addr + c * 32, o);
+        tmem_ld32(o_addr + c * 32, o);
         tmem_wait_ld();
         if (live) {
           float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
@@ -606,7 +672,7 @@ group_attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUte
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) {
+  if (warp == 9) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
   }
 }
@@ -625,15 +691,15 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [rows = N*H][hd] bf16 view, box of 64 columns x 1 row, 128-byte swizzle.
-static moga_status make_row_map(CUtensorMap* m, const void* base, int64_t rows, int hd) {
+// [rows][H][hd] bf16 viewed as 3-D {hd, H, rows}; box {64, 1, 128}, 128B swizzle.
+static moga_status make_map(CUtensorMap* m, const void* base, int64_t rows, int H, int hd) {
   auto fn = encode_fn();
   if (!fn) return fail(MOGA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  cuuint64_t gdim[2] = {(cuuint64_t)hd, (cuuint64_t)rows};
-  cuuint64_t gstride[1] = {(cuuint64_t)hd * 2};
-  cuuint32_t box[2] = {64, 1};
-  cuuint32_t estride[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estride,
+  cuuint64_t gdim[3] = {(cuuint64_t)hd, (cuuint64_t)H, (cuuint64_t)rows};
+  cuuint64_t gstride[2] = {(cuuint64_t)hd * 2, (cuuint64_t)H * hd * 2};
+  cuuint32_t box[3] = {64, 1, BM};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box, estride,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MOGA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -646,42 +712,66 @@ static long long default_timeout_cycles() {
 }
 
 template <int HD>
-static moga_status launch(const Params& prm, int grid, const void* q, const void* k, const void* v,
-                          cudaStream_t s) {
+static moga_status launch_attn(const Params& prm, int grid, const void* q, const void* k, const void* v,
+                               cudaStream_t s) {
   using S = SmemLayout<HD>;
-  cudaError_t e = cudaFuncSetAttribute(group_attn_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
   if (e != cudaSuccess) return fail(MOGA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
   CUtensorMap mq, mk, mv;
-  const int64_t rows = (int64_t)prm.N * prm.H;
   moga_status st;
-  if ((st = make_row_map(&mq, q, rows, HD)) != MOGA_OK) return st;
-  if ((st = make_row_map(&mk, k, rows, HD)) != MOGA_OK) return st;
-  if ((st = make_row_map(&mv, v, rows, HD)) != MOGA_OK) return st;
+  if ((st = make_map(&mq, q, prm.N, prm.H, HD)) != MOGA_OK) return st;
+  if ((st = make_map(&mk, k, prm.N, prm.H, HD)) != MOGA_OK) return st;
+  if ((st = make_map(&mv, v, prm.N, prm.H, HD)) != MOGA_OK) return st;
   if (grid <= 0) return MOGA_OK;
-  group_attn_kernel<HD><<<grid, kThreads, S::kBytes, s>>>(prm, mq, mk, mv);
-  return check_launch("group attention kernel");
+  attn_kernel<HD><<<grid, kThreads, S::kBytes, s>>>(prm, mq, mk, mv);
+  return check_launch("attention kernel");
 }
 
+static moga_status launch_gather(const Params& prm, int hd, const void* q, const void* k, const void* v, void* ws,
+                                 cudaStream_t s) {
+  const size_t bytes = (size_t)prm.N * prm.H * hd * 2;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const int row_u4 = prm.H * hd / 8;
+  const int grid = ceil_div(prm.N, 8);
+  const uint4 *qs = static_cast<const uint4*>(q), *ks = static_cast<const uint4*>(k),
+              *vs = static_cast<const uint4*>(v);
+  uint4 *qd = reinterpret_cast<uint4*>(w), *kd = reinterpret_cast<uint4*>(w + bytes),
+        *vd = reinterpret_cast<uint4*>(w + 2 * bytes);
+  if (prm.mode == MODE_MOGA)
+    gather3_kernel<MODE_MOGA><<<grid, 256, 0, s>>>(prm, qs, ks, vs, qd, kd, vd, row_u4);
+  else
+    gather3_kernel<MODE_WINDOW><<<grid, 256, 0, s>>>(prm, qs, ks, vs, qd, kd, vd, row_u4);
+  return check_launch("gather kernel");
+}
+
+static moga_status dispatch_attn(const Params& prm, int grid, int hd, const void* q, const void* k, const void* v,
+                                 cudaStream_t s) {
+  return hd == 128 ? launch_attn<128>(prm, grid, q, k, v, s) : launch_attn<64>(prm, grid, q, k, v, s);
+}
+
+static size_t attn_ws_bytes(int64_t N, int H, int hd) { return 3 * (size_t)N * H * hd * 2; }
+
 static moga_status check_common(const void* q, const void* k, const void* v, int64_t N, int H, int hd,
-                                const float* o_acc, const char* who) {
+                                const float* o_acc, const void* ws, size_t ws_bytes, bool need_ws, const char* who) {
   if (!q || !k || !v || !o_acc) return fail(MOGA_ERR_INVALID_ARG, "%s: null pointer", who);
   if (N <= 0 || H <= 0 || N * (int64_t)H >= INT32_MAX) return fail(MOGA_ERR_INVALID_ARG, "%s: N*H out of range", who);
   if (hd != 64 && hd != 128) return fail(MOGA_ERR_UNSUPPORTED, "%s: head_dim %d (supported: 64, 128)", who, hd);
   const uintptr_t a = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
-                      reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o_acc);
+                      reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o_acc) |
+                      reinterpret_cast<uintptr_t>(ws);
   if (a & 15) return fail(MOGA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+  if (need_ws) {
+    if (!ws) return fail(MOGA_ERR_INVALID_ARG, "%s: null workspace", who);
+    if (ws_bytes < attn_ws_bytes(N, H, hd))
+      return fail(MOGA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", who, ws_bytes, attn_ws_bytes(N, H, hd));
+  }
   return MOGA_OK;
-}
-
-static moga_status dispatch(const Params& prm, int grid, int hd, const void* q, const void* k, const void* v,
-                            cudaStream_t s) {
-  return hd == 128 ? launch<128>(prm, grid, q, k, v, s) : launch<64>(prm, grid, q, k, v, s);
 }
 
 // Temporal groups of the static window branch (as-equal-as-possible runs of
 // at most tg_max frames inside each shot, longer runs first; adjacent-shot
 // frames on the K/V side at each cut).
-static moga_status build_temporal_groups(const moga_stga_geom& g, std::vector<TGroup>& out) {
+static void build_temporal_groups(const moga_stga_geom& g, std::vector<TGroup>& out) {
   int start = 0;
   for (int s = 0; s < g.n_shots; ++s) {
     const int len = g.shot_len[s];
@@ -698,7 +788,6 @@ static moga_status build_temporal_groups(const moga_stga_geom& g, std::vector<TG
     }
     start += len;
   }
-  return MOGA_OK;
 }
 
 }  // namespace attn
@@ -707,8 +796,8 @@ static moga_status build_temporal_groups(const moga_stga_geom& g, std::vector<TG
 using namespace moga;
 using namespace moga::attn;
 
-// Test hook (not declared in the public header): bounded-wait timeout in SM
-// cycles and debug flags for the next group-attention launch on this thread.
+// Test hook (declared in include/moga_testing.h): bounded-wait limit in SM
+// cycles and debug flags for the next attention launches on this thread.
 static thread_local long long t_timeout_override = 0;
 static thread_local int t_debug_flags = 0;
 extern "C" void moga_test_set_attn_debug(long long timeout_cycles, int flags) {
@@ -721,10 +810,16 @@ static void fill_debug(Params& prm) {
   prm.debug_flags = t_debug_flags;
 }
 
+extern "C" size_t moga_attn_ws_bytes(int64_t N, int32_t H, int32_t hd) {
+  if (N <= 0 || H <= 0 || (hd != 64 && hd != 128) || N * (int64_t)H >= INT32_MAX) return 0;
+  return attn_ws_bytes(N, H, hd);
+}
+
 extern "C" moga_status moga_group_attn(const void* q, const void* k, const void* v, int64_t N, int32_t H, int32_t hd,
                                        const int32_t* perm, const int32_t* cu_seqlens, int32_t M,
-                                       const float* gate_prob, float softmax_scale, float* o_acc, void* stream) {
-  moga_status st = check_common(q, k, v, N, H, hd, o_acc, "moga_group_attn");
+                                       const float* gate_prob, float softmax_scale, float* o_acc, void* ws,
+                                       size_t ws_bytes, void* stream) {
+  moga_status st = check_common(q, k, v, N, H, hd, o_acc, ws, ws_bytes, true, "moga_group_attn");
   if (st != MOGA_OK) return st;
   if (!perm || !cu_seqlens || !gate_prob) return fail(MOGA_ERR_INVALID_ARG, "moga_group_attn: null pointer");
   if (M < 1 || M > 32) return fail(MOGA_ERR_INVALID_ARG, "moga_group_attn: M=%d not in [1, 32]", M);
@@ -741,13 +836,18 @@ extern "C" moga_status moga_group_attn(const void* q, const void* k, const void*
   prm.gate = gate_prob;
   prm.o_acc = o_acc;
   fill_debug(prm);
-  // upper bound on the tile count: sum_i ceil(n_i / BM) <= N / BM + M
-  const int grid = (ceil_div((int)N, BM) + M) * H;
-  return dispatch(prm, grid, hd, q, k, v, static_cast<cudaStream_t>(stream));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = launch_gather(prm, hd, q, k, v, ws, s)) != MOGA_OK) return st;
+  const uint8_t* w = static_cast<const uint8_t*>(ws);
+  const size_t bytes = (size_t)N * H * hd * 2;
+  // upper bound on the CTA count: sum_i ceil(n_i / 256) <= N / 256 + M
+  const int grid = (ceil_div((int)N, 2 * BM) + M) * H;
+  return dispatch_attn(prm, grid, hd, w, w + bytes, w + 2 * bytes, s);
 }
 
 extern "C" moga_status stga_attn(const void* q, const void* k, const void* v, int32_t H, int32_t hd,
-                                 const moga_stga_geom* geom, float softmax_scale, float* o_acc, void* stream) {
+                                 const moga_stga_geom* geom, float softmax_scale, float* o_acc, void* ws,
+                                 size_t ws_bytes, void* stream) {
   if (!geom || !geom->shot_len) return fail(MOGA_ERR_INVALID_ARG, "stga_attn: null geometry");
   const moga_stga_geom& g = *geom;
   if (g.T <= 0 || g.h <= 0 || g.w <= 0 || g.win_h <= 0 || g.win_w <= 0 || g.n_shots <= 0 || g.tg_max < 0 ||
@@ -761,7 +861,7 @@ extern "C" moga_status stga_attn(const void* q, const void* k, const void* v, in
   }
   if (tsum != g.T) return fail(MOGA_ERR_INVALID_ARG, "stga_attn: shot lengths sum to %lld, T=%d", tsum, g.T);
   const int64_t N = (int64_t)g.T * g.h * g.w;
-  moga_status st = check_common(q, k, v, N, H, hd, o_acc, "stga_attn");
+  moga_status st = check_common(q, k, v, N, H, hd, o_acc, ws, ws_bytes, true, "stga_attn");
   if (st != MOGA_OK) return st;
   if (!(softmax_scale > 0.f)) return fail(MOGA_ERR_INVALID_ARG, "stga_attn: softmax_scale must be > 0");
   std::vector<TGroup> tgs;
@@ -788,15 +888,19 @@ extern "C" moga_status stga_attn(const void* q, const void* k, const void* v, in
   prm.tg_tiles[0] = 0;
   for (int i = 0; i < prm.n_tg; ++i) {
     prm.tg[i] = tgs[i];
-    const int qt = ceil_div((tgs[i].t1 - tgs[i].t0) * prm.whw, BM);
-    prm.tg_tiles[i + 1] = prm.tg_tiles[i] + prm.n_win * H * qt;
+    const int qp = ceil_div((tgs[i].t1 - tgs[i].t0) * prm.whw, 2 * BM);
+    prm.tg_tiles[i + 1] = prm.tg_tiles[i] + prm.n_win * H * qp;
   }
   fill_debug(prm);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // window groups, then frames: both add into o_acc; stream order keeps them apart
+  // window groups (gathered into window-major order), then frames (already
+  // contiguous); both add into o_acc and stream order keeps them apart
   prm.mode = MODE_WINDOW;
-  st = dispatch(prm, prm.tg_tiles[prm.n_tg], hd, q, k, v, s);
+  if ((st = launch_gather(prm, hd, q, k, v, ws, s)) != MOGA_OK) return st;
+  const uint8_t* w = static_cast<const uint8_t*>(ws);
+  const size_t bytes = (size_t)N * H * hd * 2;
+  st = dispatch_attn(prm, prm.tg_tiles[prm.n_tg], hd, w, w + bytes, w + 2 * bytes, s);
   if (st != MOGA_OK) return st;
   prm.mode = MODE_FRAME;
-  return dispatch(prm, g.T * H * ceil_div(prm.hw, BM), hd, q, k, v, s);
+  return dispatch_attn(prm, g.T * H * ceil_div(prm.hw, 2 * BM), hd, q, k, v, s);
 }

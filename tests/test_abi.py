@@ -65,13 +65,19 @@ def test_permute_argument_checks(lib):
 
 
 def test_attention_argument_checks(lib):
-    assert lib.moga_group_attn(FAKE, FAKE, FAKE, 100, 2, 96, FAKE, FAKE, 4, FAKE, 0.1, FAKE, None) == 2
+    W = 1 << 40
+    ga = lambda *a: lib.moga_group_attn(*a)  # noqa: E731
+    assert ga(FAKE, FAKE, FAKE, 100, 2, 96, FAKE, FAKE, 4, FAKE, 0.1, FAKE, FAKE, W, None) == 2
     assert b"head_dim" in lib.moga_last_error()
-    assert lib.moga_group_attn(FAKE, FAKE, FAKE, 100, 2, 128, FAKE, FAKE, 40, FAKE, 0.1, FAKE, None) == 1
-    assert lib.moga_group_attn(FAKE, FAKE, FAKE, 100, 2, 128, FAKE, FAKE, 4, FAKE, -1.0, FAKE, None) == 1
-    assert lib.moga_group_attn(FAKE, FAKE, FAKE, 1 << 30, 4, 128, FAKE, FAKE, 4, FAKE, 0.1, FAKE, None) == 1
+    assert ga(FAKE, FAKE, FAKE, 100, 2, 128, FAKE, FAKE, 40, FAKE, 0.1, FAKE, FAKE, W, None) == 1
+    assert ga(FAKE, FAKE, FAKE, 100, 2, 128, FAKE, FAKE, 4, FAKE, -1.0, FAKE, FAKE, W, None) == 1
+    assert ga(FAKE, FAKE, FAKE, 1 << 30, 4, 128, FAKE, FAKE, 4, FAKE, 0.1, FAKE, FAKE, W, None) == 1
     mis = ctypes.c_void_p(4096 + 8)
-    assert lib.moga_group_attn(mis, FAKE, FAKE, 100, 2, 128, FAKE, FAKE, 4, FAKE, 0.1, FAKE, None) == 1
+    assert ga(mis, FAKE, FAKE, 100, 2, 128, FAKE, FAKE, 4, FAKE, 0.1, FAKE, FAKE, W, None) == 1
+    assert ga(FAKE, FAKE, FAKE, 100, 2, 128, FAKE, FAKE, 4, FAKE, 0.1, FAKE, FAKE, 1000, None) == 3
+    assert ga(FAKE, FAKE, FAKE, 100, 2, 128, FAKE, FAKE, 4, FAKE, 0.1, FAKE, None, W, None) == 1
+    assert lib.moga_attn_ws_bytes(100, 2, 128) == 3 * 100 * 2 * 128 * 2
+    assert lib.moga_attn_ws_bytes(100, 2, 96) == 0
 
 
 def _geom(**kw):
@@ -88,7 +94,7 @@ def _geom(**kw):
 ])
 def test_stga_geometry_checks(lib, bad, msg):
     s, keep = _geom_struct(_geom(**bad))
-    st = lib.stga_attn(FAKE, FAKE, FAKE, 2, 128, ctypes.byref(s), 0.1, FAKE, None)
+    st = lib.stga_attn(FAKE, FAKE, FAKE, 2, 128, ctypes.byref(s), 0.1, FAKE, FAKE, 1 << 40, None)
     assert st == 1 and msg in lib.moga_last_error(), lib.moga_last_error()
 
 
