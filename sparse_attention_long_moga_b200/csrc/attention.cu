@@ -199,6 +199,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
       : "memory");
 }
 
+// 32 lanes x 8 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 // 32 lanes x 16 consecutive 32-bit columns.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
   asm volatile(
@@ -216,6 +223,29 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe, used for a quarter of the softmax exponentials so the
+// SFU (ex2) and the FMA pipe share the load.  Method: x = n + f with n the
+// nearest integer (taken from the low mantissa bits of x + 1.5*2^23) and
+// f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose coefficients were fitted
+// here by iteratively reweighted least squares on the relative error
+// (max relative error 7.5e-5 on [-1/2, 1/2], below the bf16 rounding of P);
+// 2^n is added into the exponent field.  x is clamped to >= -126 so the
+// exponent never wraps (2^-126 is negligible next to the row sum >= 1).
+#ifndef MOGA_POLY_EXP2
+#define MOGA_POLY_EXP2 0
+#endif
+constexpr float kExp2C0 = 0.99992806f;
+constexpr float kExp2C1 = 0.69326097f;
+constexpr float kExp2C2 = 0.24261114f;
+constexpr float kExp2C3 = 0.05517166f;
+__device__ __forceinline__ float poly_exp2(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -264,54 +294,65 @@ __device__ __forceinline__ int token_of(const Params& p, int idx) {
 
 struct Tile {
   int head, q_begin, q_end, kv_begin, kv_end;
-  int valid;  // 0: this CTA has no work
+  int valid;  // 0: past the last tile
 };
 
-// Decode blockIdx into a tile pair (thread 0 only; shared through smem).
-__device__ void decode_tile(const Params& p, int L, Tile& t) {
+// MoGA groups in processing order (largest first), built once per CTA.
+struct GroupTable {
+  int n;
+  int start[32], size[32];
+  int prefix[33];   // CTA-tile prefix over the ordered groups
+};
+
+__device__ void build_group_table(const Params& p, GroupTable& gt) {
+  int size[32], order[32];
+  for (int i = 0; i < p.M; ++i) {
+    size[i] = __ldg(p.cu + i + 1) - __ldg(p.cu + i);
+    order[i] = i;
+  }
+  for (int i = 1; i < p.M; ++i) {   // insertion sort, descending size, stable
+    const int o = order[i];
+    int j = i - 1;
+    while (j >= 0 && size[order[j]] < size[o]) {
+      order[j + 1] = order[j];
+      --j;
+    }
+    order[j + 1] = o;
+  }
+  gt.n = p.M;
+  gt.prefix[0] = 0;
+  for (int k = 0; k < p.M; ++k) {
+    const int g = order[k];
+    gt.start[k] = __ldg(p.cu + g);
+    gt.size[k] = size[g];
+    gt.prefix[k + 1] = gt.prefix[k] + ceil_div(size[g], 2 * BM) * p.H;
+  }
+}
+
+// Tile L (a pair of 128-row query tiles of one group and head).  Tiles are
+// ordered so that consecutive ones share a group's K/V through L2.
+__device__ __forceinline__ Tile decode_tile(const Params& p, const GroupTable& gt, int L) {
+  Tile t;
   t.valid = 0;
   constexpr int kPair = 2 * BM;
   if (p.mode == MODE_MOGA) {
-    // largest groups first, then head, then query-tile pair (K/V of one group
-    // and head are reused by consecutive CTAs through L2)
-    int size[32], order[32];
-    for (int i = 0; i < p.M; ++i) {
-      size[i] = __ldg(p.cu + i + 1) - __ldg(p.cu + i);
-      order[i] = i;
-    }
-    for (int i = 1; i < p.M; ++i) {
-      const int o = order[i];
-      int j = i - 1;
-      while (j >= 0 && size[order[j]] < size[o]) {
-        order[j + 1] = order[j];
-        --j;
-      }
-      order[j + 1] = o;
-    }
-    int rem = L;
-    for (int k = 0; k < p.M; ++k) {
-      const int g = order[k];
-      const int qp = ceil_div(size[g], kPair);
-      const int n = qp * p.H;
-      if (rem < n) {
-        const int start = __ldg(p.cu + g);
-        t.head = rem / qp;
-        const int qi = rem - t.head * qp;
-        t.q_begin = start + qi * kPair;
-        t.q_end = min(start + size[g], t.q_begin + kPair);
-        t.kv_begin = start;
-        t.kv_end = start + size[g];
-        t.valid = 1;
-        return;
-      }
-      rem -= n;
-    }
-    return;
+    if (L >= gt.prefix[gt.n]) return t;
+    int k = 0;
+    while (gt.prefix[k + 1] <= L) ++k;
+    const int qp = ceil_div(gt.size[k], kPair);
+    const int rem = L - gt.prefix[k];
+    t.head = rem / qp;
+    const int qi = rem - t.head * qp;
+    t.q_begin = gt.start[k] + qi * kPair;
+    t.q_end = min(gt.start[k] + gt.size[k], t.q_begin + kPair);
+    t.kv_begin = gt.start[k];
+    t.kv_end = gt.start[k] + gt.size[k];
+    t.valid = 1;
+    return t;
   }
   if (p.mode == MODE_FRAME) {
     const int qp = ceil_div(p.hw, kPair);
-    const int total = p.T * p.H * qp;
-    if (L >= total) return;
+    if (L >= p.T * p.H * qp) return t;
     const int frame = L / (p.H * qp);
     const int rem = L - frame * p.H * qp;
     t.head = rem / qp;
@@ -321,10 +362,10 @@ __device__ void decode_tile(const Params& p, int L, Tile& t) {
     t.q_begin = t.kv_begin + qi * kPair;
     t.q_end = min(t.kv_end, t.q_begin + kPair);
     t.valid = 1;
-    return;
+    return t;
   }
   // window groups: temporal group, window, head, query-tile pair
-  if (L >= p.tg_tiles[p.n_tg]) return;
+  if (L >= p.tg_tiles[p.n_tg]) return t;
   int g = 0;
   while (p.tg_tiles[g + 1] <= L) ++g;
   const TGroup tg = p.tg[g];
@@ -341,6 +382,7 @@ __device__ void decode_tile(const Params& p, int L, Tile& t) {
   t.kv_begin = (base + tg.t0 - tg.a_prev) * p.whw;
   t.kv_end = (base + tg.t1 + tg.a_next) * p.whw;
   t.valid = 1;
+  return t;
 }
 
 // ------------------------------------------------------------------ gather
@@ -377,9 +419,10 @@ struct SmemLayout {
   static constexpr int kK0 = kQ + 2 * kTileBytes;           // two K stages
   static constexpr int kV0 = kK0 + 2 * kTileBytes;          // two V stages
   static constexpr int kBar = kV0 + 2 * kTileBytes;
-  static constexpr int kNumBars = 16;
+  static constexpr int kNumBars = 24;
   static constexpr int kMisc = kBar + kNumBars * 8;
-  static constexpr int kEnd = kMisc + 64;
+  static constexpr int kTable = kMisc + 64;
+  static constexpr int kEnd = kTable + (int)sizeof(GroupTable);
   // 1 KB slack to align the dynamic base to 1024 bytes; the hd = 64 layout is
   // padded so that two CTAs never share an SM (each holds all 512 TMEM columns)
   static constexpr int kBytes = (HD == 64 ? 120 * 1024 : kEnd) + 1024;
@@ -387,20 +430,28 @@ struct SmemLayout {
 
 enum Bar : int {
   B_FULL_Q = 0,
-  B_FULL_K = 1,   // +stage
-  B_FULL_V = 3,   // +stage
-  B_EMPTY_K = 5,  // +stage
-  B_EMPTY_V = 7,  // +stage
-  B_S_FULL = 9,   // +query tile
-  B_P_FULL = 11,  // +query tile
-  B_O_FULL = 13,
-  B_MMA_END = 14
+  B_EMPTY_Q = 1,
+  B_FULL_K = 2,   // +stage
+  B_FULL_V = 4,   // +stage
+  B_EMPTY_K = 6,  // +stage
+  B_EMPTY_V = 8,  // +stage
+  B_S_FULL = 10,  // +query tile
+  B_P_FULL = 12,  // +query tile
+  B_O_FULL = 14,  // +query tile
+  B_O_EMPTY = 16, // +query tile
+  B_MMA_END = 18,
+  B_COUNT = 19
 };
 
 // ------------------------------------------------------------------ the kernel
 
+// Persistent: CTA b processes tiles b, b + gridDim.x, ...  Barrier phases run
+// on across tiles (counters below); TMEM is allocated once.  The producer
+// loads the next tile's Q as soon as the last S MMA of the current tile has
+// read Q, and the MMA warp starts the next tile's S products while the
+// softmax warps are still writing the current tile's output.
 template <int HD>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 1)
 attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tm_q,
             const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
   using S = SmemLayout<HD>;
@@ -411,16 +462,15 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
   int* misc = reinterpret_cast<int*>(smem + S::kMisc);
   volatile int* abort_flag = misc + 0;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 1);
-  Tile* tile_sh = reinterpret_cast<Tile*>(misc + 4);
+  GroupTable* gt_sh = reinterpret_cast<GroupTable*>(smem + S::kTable);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    Tile t;
-    decode_tile(p, blockIdx.x, t);
-    *tile_sh = t;
     *abort_flag = 0;
+    if (p.mode == MODE_MOGA) build_group_table(p, *gt_sh);
     mbar_init(bar(B_FULL_Q), 1);
+    mbar_init(bar(B_EMPTY_Q), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(B_FULL_K + s), 1);
       mbar_init(bar(B_FULL_V + s), 1);
@@ -428,15 +478,15 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
       mbar_init(bar(B_EMPTY_V + s), 1);
       mbar_init(bar(B_S_FULL + s), 1);
       mbar_init(bar(B_P_FULL + s), BM);
+      mbar_init(bar(B_O_FULL + s), 1);
+      mbar_init(bar(B_O_EMPTY + s), BM);
     }
-    mbar_init(bar(B_O_FULL), 1);
     mbar_init(bar(B_MMA_END), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  const Tile t = *tile_sh;
-  if (!t.valid) return;   // uniform across the CTA
-  const bool has_q1 = t.q_begin + BM < t.q_end;
+  const GroupTable& gt = *gt_sh;
+  if (!decode_tile(p, gt, blockIdx.x).valid) return;   // uniform: this CTA has no tile
 
   if (warp == 9) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -449,45 +499,55 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const long long timeout = p.timeout_cycles;
-  const int n_kv = ceil_div(t.kv_end - t.kv_begin, BN);
 
   if (warp == 8) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       const bool skip_q = (p.debug_flags & 1) != 0;
-      int issued_k[2] = {-1, -1}, issued_v[2] = {-1, -1};
-      if (!skip_q) {
-        mbar_arrive_expect_tx(bar(B_FULL_Q), (has_q1 ? 2 : 1) * S::kTileBytes);
-        for (int qt = 0; qt < (has_q1 ? 2 : 1); ++qt)
+      int last_k[2] = {-1, -1}, last_v[2] = {-1, -1}, last_q = -1;
+      int c = 0;   // K/V tiles issued so far (ring position)
+      bool ok = true;
+      for (int i = 0, L = blockIdx.x; ok; ++i, L += gridDim.x) {
+        const Tile t = decode_tile(p, gt, L);
+        if (!t.valid) break;
+        const bool has_q1 = t.q_begin + BM < t.q_end;
+        // Q of the previous tile has been read by its last S product
+        if (!(ok = mbar_wait(bar(B_EMPTY_Q), (i & 1) ^ 1, abort_flag, timeout))) break;
+        if (!skip_q) {
+          mbar_arrive_expect_tx(bar(B_FULL_Q), (has_q1 ? 2 : 1) * S::kTileBytes);
+          for (int qt = 0; qt < (has_q1 ? 2 : 1); ++qt)
+#pragma unroll
+            for (int hh = 0; hh < S::kHalves; ++hh)
+              tma_load_3d(sbase + S::kQ + qt * S::kTileBytes + hh * kHalfBytes, &tm_q, hh * 64, t.head,
+                          t.q_begin + qt * BM, bar(B_FULL_Q));
+          last_q = i;
+        }
+        const int n_kv = ceil_div(t.kv_end - t.kv_begin, BN);
+        for (int j = 0; j < n_kv; ++j, ++c) {
+          const int st = c & 1;
+          const uint32_t ph = (c >> 1) & 1;
+          const int row = t.kv_begin + j * BN;
+          if (!(ok = mbar_wait(bar(B_EMPTY_K + st), ph ^ 1, abort_flag, timeout))) break;
+          mbar_arrive_expect_tx(bar(B_FULL_K + st), S::kTileBytes);
 #pragma unroll
           for (int hh = 0; hh < S::kHalves; ++hh)
-            tma_load_3d(sbase + S::kQ + qt * S::kTileBytes + hh * kHalfBytes, &tm_q, hh * 64, t.head,
-                        t.q_begin + qt * BM, bar(B_FULL_Q));
-      }
-      for (int j = 0; j < n_kv; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        const int row = t.kv_begin + j * BN;
-        if (!mbar_wait(bar(B_EMPTY_K + st), ph ^ 1, abort_flag, timeout)) break;
-        mbar_arrive_expect_tx(bar(B_FULL_K + st), S::kTileBytes);
+            tma_load_3d(sbase + S::kK0 + st * S::kTileBytes + hh * kHalfBytes, &tm_k, hh * 64, t.head, row,
+                        bar(B_FULL_K + st));
+          last_k[st] = c;
+          if (!(ok = mbar_wait(bar(B_EMPTY_V + st), ph ^ 1, abort_flag, timeout))) break;
+          mbar_arrive_expect_tx(bar(B_FULL_V + st), S::kTileBytes);
 #pragma unroll
-        for (int hh = 0; hh < S::kHalves; ++hh)
-          tma_load_3d(sbase + S::kK0 + st * S::kTileBytes + hh * kHalfBytes, &tm_k, hh * 64, t.head, row,
-                      bar(B_FULL_K + st));
-        issued_k[st] = j;
-        if (!mbar_wait(bar(B_EMPTY_V + st), ph ^ 1, abort_flag, timeout)) break;
-        mbar_arrive_expect_tx(bar(B_FULL_V + st), S::kTileBytes);
-#pragma unroll
-        for (int hh = 0; hh < S::kHalves; ++hh)
-          tma_load_3d(sbase + S::kV0 + st * S::kTileBytes + hh * kHalfBytes, &tm_v, hh * 64, t.head, row,
-                      bar(B_FULL_V + st));
-        issued_v[st] = j;
+          for (int hh = 0; hh < S::kHalves; ++hh)
+            tma_load_3d(sbase + S::kV0 + st * S::kTileBytes + hh * kHalfBytes, &tm_v, hh * 64, t.head, row,
+                        bar(B_FULL_V + st));
+          last_v[st] = c;
+        }
       }
       // let every copy started here land before the CTA can exit
-      if (!skip_q) mbar_drain(bar(B_FULL_Q), 0, timeout);
+      if (last_q >= 0) mbar_drain(bar(B_FULL_Q), last_q & 1, timeout);
       for (int st = 0; st < 2; ++st) {
-        if (issued_k[st] >= 0) mbar_drain(bar(B_FULL_K + st), (issued_k[st] >> 1) & 1, timeout);
-        if (issued_v[st] >= 0) mbar_drain(bar(B_FULL_V + st), (issued_v[st] >> 1) & 1, timeout);
+        if (last_k[st] >= 0) mbar_drain(bar(B_FULL_K + st), (last_k[st] >> 1) & 1, timeout);
+        if (last_v[st] >= 0) mbar_drain(bar(B_FULL_V + st), (last_v[st] >> 1) & 1, timeout);
       }
     }
     __syncwarp();
@@ -498,10 +558,12 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
       constexpr uint32_t idesc_pv = instr_desc(HD, true);
       const uint32_t tmem_s[2] = {tmem, tmem + 128};
       const uint32_t tmem_o[2] = {tmem + 256, tmem + 384};
-      const int nq = has_q1 ? 2 : 1;
-      auto issue_s = [&](int qt, int j) {
+      int c = 0;                   // K/V ring position
+      int pc[2] = {0, 0};          // P tiles consumed per query tile
+      int oc[2] = {0, 0};          // outputs produced per query tile
+      auto issue_s = [&](int qt, int cc) {
         const uint32_t qa = sbase + S::kQ + qt * S::kTileBytes;
-        const uint32_t ka = sbase + S::kK0 + (j & 1) * S::kTileBytes;
+        const uint32_t ka = sbase + S::kK0 + (cc & 1) * S::kTileBytes;
 #pragma unroll
         for (int ks = 0; ks < HD / 16; ++ks) {
           const uint64_t ad = smem_desc(qa + (ks >> 2) * kHalfBytes + (ks & 3) * 32, 16, 1024);
@@ -510,55 +572,67 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
         }
         tc_commit(bar(B_S_FULL + qt));
       };
-      auto issue_pv = [&](int qt, int j) {
-        const uint32_t va = sbase + S::kV0 + (j & 1) * S::kTileBytes;
+      auto issue_pv = [&](int qt, int cc, bool acc) {
+        const uint32_t va = sbase + S::kV0 + (cc & 1) * S::kTileBytes;
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks) {
           const uint64_t bd = smem_desc(va + ks * 16 * 128, kHalfBytes, 1024);
-          tc_mma_ts(tmem_o[qt], tmem_s[qt] + ks * 8, bd, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+          tc_mma_ts(tmem_o[qt], tmem_s[qt] + ks * 8, bd, idesc_pv, (acc || ks > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(bar(B_FULL_Q), 0, abort_flag, timeout) &&
-                mbar_wait(bar(B_FULL_K + 0), 0, abort_flag, timeout);
-      if (ok) {
-        tc_fence_after();
-        for (int qt = 0; qt < nq; ++qt) issue_s(qt, 0);
-        tc_commit(bar(B_EMPTY_K + 0));
-      }
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        const bool more = j + 1 < n_kv;
-        ok = mbar_wait(bar(B_FULL_V + st), ph, abort_flag, timeout) &&
-             mbar_wait(bar(B_P_FULL + 0), j & 1, abort_flag, timeout);
+      bool ok = true;
+      for (int i = 0, L = blockIdx.x; ok; ++i, L += gridDim.x) {
+        const Tile t = decode_tile(p, gt, L);
+        if (!t.valid) break;
+        const bool has_q1 = t.q_begin + BM < t.q_end;
+        const int nq = has_q1 ? 2 : 1;
+        const int n_kv = ceil_div(t.kv_end - t.kv_begin, BN);
+        ok = mbar_wait(bar(B_FULL_Q), i & 1, abort_flag, timeout) &&
+             mbar_wait(bar(B_FULL_K + (c & 1)), (c >> 1) & 1, abort_flag, timeout);
         if (!ok) break;
         tc_fence_after();
-        issue_pv(0, j);
-        if (more) {
-          ok = mbar_wait(bar(B_FULL_K + ((j + 1) & 1)), ((j + 1) >> 1) & 1, abort_flag, timeout);
+        for (int qt = 0; qt < nq; ++qt) issue_s(qt, c);
+        if (n_kv == 1) tc_commit(bar(B_EMPTY_Q));
+        tc_commit(bar(B_EMPTY_K + (c & 1)));
+        for (int j = 0; j < n_kv; ++j, ++c) {
+          const int st = c & 1;
+          const uint32_t ph = (c >> 1) & 1;
+          const bool more = j + 1 < n_kv;
+          for (int qt = 0; qt < nq; ++qt) {
+            // the first P.V of a tile overwrites O: the epilogue of this query
+            // tile's previous output must have read it
+            if (j == 0 && !(ok = mbar_wait(bar(B_O_EMPTY + qt), (oc[qt] & 1) ^ 1, abort_flag, timeout))) break;
+            if (qt == 0 && !(ok = mbar_wait(bar(B_FULL_V + st), ph, abort_flag, timeout))) break;
+            if (!(ok = mbar_wait(bar(B_P_FULL + qt), pc[qt] & 1, abort_flag, timeout))) break;
+            tc_fence_after();
+            issue_pv(qt, c, j > 0);
+            ++pc[qt];
+            if (qt == 0 && more) {
+              if (!(ok = mbar_wait(bar(B_FULL_K + ((c + 1) & 1)), ((c + 1) >> 1) & 1, abort_flag, timeout))) break;
+              tc_fence_after();
+              issue_s(0, c + 1);
+            }
+          }
           if (!ok) break;
-          tc_fence_after();
-          issue_s(0, j + 1);
+          tc_commit(bar(B_EMPTY_V + st));
+          if (more) {
+            if (has_q1) issue_s(1, c + 1);
+            if (j + 2 == n_kv) tc_commit(bar(B_EMPTY_Q));   // last S products of this tile issued
+            tc_commit(bar(B_EMPTY_K + ((c + 1) & 1)));
+          }
         }
-        if (has_q1) {
-          ok = mbar_wait(bar(B_P_FULL + 1), j & 1, abort_flag, timeout);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(1, j);
-        }
-        tc_commit(bar(B_EMPTY_V + st));
-        if (more) {
-          if (has_q1) issue_s(1, j + 1);
-          tc_commit(bar(B_EMPTY_K + ((j + 1) & 1)));
+        if (!ok) break;
+        for (int qt = 0; qt < nq; ++qt) {
+          tc_commit(bar(B_O_FULL + qt));
+          ++oc[qt];
         }
       }
-      if (ok) tc_commit(bar(B_O_FULL));
       // every MMA issued here has finished before TMEM is released
       tc_commit(bar(B_MMA_END));
       mbar_drain(bar(B_MMA_END), 0, timeout);
     }
     __syncwarp();
-  } else if (warp < 4 || has_q1) {
+  } else {
     // ---------------------------------------------------------------- softmax
     const int qt = warp >> 2;                            // query tile of this warpgroup
     const int row = (warp & 3) * 32 + lane;              // TMEM lane == query row
@@ -566,103 +640,112 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
     const uint32_t s_addr = tmem + lane_addr + qt * 128;
     const uint32_t o_addr = tmem + lane_addr + 256 + qt * 128;
     const float sl = p.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;
+    int sc = 0, oc = 0;   // S tiles and outputs handled by this warpgroup
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + qt), j & 1, abort_flag, timeout));
-      if (!ok) break;
-      tc_fence_after();
-      float s[BN];
+    for (int L = blockIdx.x; ok; L += gridDim.x) {
+      const Tile t = decode_tile(p, gt, L);
+      if (!t.valid) break;
+      if (qt == 1 && !(t.q_begin + BM < t.q_end)) continue;   // no second query tile here
+      const int n_kv = ceil_div(t.kv_end - t.kv_begin, BN);
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < n_kv; ++j, ++sc) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + qt), sc & 1, abort_flag, timeout));
+        if (!ok) break;
+        tc_fence_after();
+        float s[BN];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(s_addr + c * 32, s + c * 32);
-      tmem_wait_ld();
-      const int valid = t.kv_end - (t.kv_begin + j * BN);
-      if (valid < BN) {
+        for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(s_addr + cc * 32, s + cc * 32);
+        tmem_wait_ld();
+        const int valid = t.kv_end - (t.kv_begin + j * BN);
+        if (valid < BN) {
 #pragma unroll
-        for (int c = 0; c < BN; ++c)
-          if (c >= valid) s[c] = -INFINITY;
-      }
-      float mx = s[0];
+          for (int cc = 0; cc < BN; ++cc)
+            if (cc >= valid) s[cc] = -INFINITY;
+        }
+        // row max with 8 independent chains (a single chain would expose the
+        // max latency 127 times)
+        float mp[8];
 #pragma unroll
-      for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
-      const float m_new = fmaxf(m_run, mx * sl);
-      if (j == 0) {
-        m_run = m_new;
-      } else {
-        // P.V of tile j-1 finished before S of tile j (issue order), so O may
-        // be rescaled here
-        const bool need = m_new > m_run + 8.0f;
+        for (int e = 0; e < 8; ++e) mp[e] = s[e];
+#pragma unroll
+        for (int cc = 8; cc < BN; cc += 8)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mp[e] = fmaxf(mp[e], s[cc + e]);
+        const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                               fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+        const float m_new = fmaxf(m_run, mx * sl);
+        // Move the reference max only when it grows by more than 2^8 (tile 0
+        // always sets it); rows that move it rescale O and l after P is written.
+        const bool need = j > 0 && m_new > m_run + 8.0f;
+        const float m_old = m_run;
+        if (j == 0 || need) m_run = m_new;
+        const float neg_m = -m_run;
+        float sp[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
+#pragma unroll
+        for (int cc = 0; cc < BN / 16; ++cc) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float a = fast_exp2(fmaf(s[cc * 16 + 2 * e], sl, neg_m));
+            const float xb = fmaf(s[cc * 16 + 2 * e + 1], sl, neg_m);
+            const float b = (MOGA_POLY_EXP2 && (e & 1)) ? poly_exp2(xb) : fast_exp2(xb);
+            sp[e & 3] += a + b;
+            pk[e] = pack_bf16x2(a, b);
+          }
+          // P overwrites S columns [8cc, 8cc+8), whose scores were read above
+          tmem_st8(s_addr + cc * 8, pk);
+        }
         if (__any_sync(0xffffffffu, need)) {
-          const float f = need ? fast_exp2(m_run - m_new) : 1.0f;
+          // P.V of tile j-1 finished before S of tile j (issue order), so O
+          // may be rescaled here, before P_j is released to the MMA warp
+          const float f = need ? fast_exp2(m_old - m_new) : 1.0f;
 #pragma unroll 1
-          for (int c = 0; c < HD / 32; ++c) {
+          for (int cc = 0; cc < HD / 32; ++cc) {
             float o[32];
-            tmem_ld32(o_addr + c * 32, o);
+            tmem_ld32(o_addr + cc * 32, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= f;
-            tmem_st32(o_addr + c * 32, o);
+            for (int e = 0; e < 32; ++e) o[e] *= f;
+            tmem_st32(o_addr + cc * 32, o);
           }
-          if (need) {
-            l_run *= f;
-            m_run = m_new;
-          }
+          l_run *= f;
         }
+        l_run += (sp[0] + sp[1]) + (sp[2] + sp[3]);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_P_FULL + qt));
       }
-      const float neg_m = -m_run;
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float a = fast_exp2(fmaf(s[c * 32 + 2 * i], sl, neg_m));
-          const float b = fast_exp2(fmaf(s[c * 32 + 2 * i + 1], sl, neg_m));
-          sum += a + b;
-          pk[i] = pack_bf16x2(a, b);
-        }
-        // P overwrites S columns [16c, 16c+16), whose scores were read above
-        tmem_st16(s_addr + c * 16, pk);
-      }
-      l_run += sum;
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(B_P_FULL + qt));
-    }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O_FULL), 0, abort_flag, timeout));
-    if (ok) {
+      if (!ok) break;
+      // ------------------------------------------------------------ epilogue
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O_FULL + qt), oc & 1, abort_flag, timeout));
+      if (!ok) break;
+      ++oc;
       tc_fence_after();
+      float o[HD];
+#pragma unroll
+      for (int cc = 0; cc < HD / 32; ++cc) tmem_ld32(o_addr + cc * 32, o + cc * 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(B_O_EMPTY + qt));   // O may be overwritten by the next tile now
       const int q_idx = t.q_begin + qt * BM + row;
-      const bool live = q_idx < t.q_end;
-      float scale = 0.f;
-      float* dst = nullptr;
-      if (live) {
+      if (q_idx < t.q_end) {
         const int tok = token_of(p, q_idx);
-        scale = 1.0f / l_run;
+        float scale = 1.0f / l_run;
         if (p.mode == MODE_MOGA) scale *= __ldg(p.gate + tok);
-        dst = p.o_acc + ((size_t)tok * p.H + t.head) * HD;
-      }
-#pragma unroll 1
-      for (int c = 0; c < HD / 32; ++c) {
-        float o[32];
-        tmem_ld32(o_addr + c * 32, o);
-        tmem_wait_ld();
-        if (live) {
-          float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
-          if (p.mode == MODE_MOGA) {
+        float4* d4 = reinterpret_cast<float4*>(p.o_acc + ((size_t)tok * p.H + t.head) * HD);
+        if (p.mode == MODE_MOGA) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              d4[i] = make_float4(o[4 * i] * scale, o[4 * i + 1] * scale, o[4 * i + 2] * scale, o[4 * i + 3] * scale);
-          } else {
+          for (int e = 0; e < HD / 4; ++e)
+            d4[e] = make_float4(o[4 * e] * scale, o[4 * e + 1] * scale, o[4 * e + 2] * scale, o[4 * e + 3] * scale);
+        } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              float4 a = d4[i];
-              a.x = fmaf(o[4 * i], scale, a.x);
-              a.y = fmaf(o[4 * i + 1], scale, a.y);
-              a.z = fmaf(o[4 * i + 2], scale, a.z);
-              a.w = fmaf(o[4 * i + 3], scale, a.w);
-              d4[i] = a;
-            }
+          for (int e = 0; e < HD / 4; ++e) {
+            float4 a = d4[e];
+            a.x = fmaf(o[4 * e], scale, a.x);
+            a.y = fmaf(o[4 * e + 1], scale, a.y);
+            a.z = fmaf(o[4 * e + 2], scale, a.z);
+            a.w = fmaf(o[4 * e + 3], scale, a.w);
+            d4[e] = a;
           }
         }
       }
@@ -744,8 +827,18 @@ static moga_status launch_gather(const Params& prm, int hd, const void* q, const
   return check_launch("gather kernel");
 }
 
-static moga_status dispatch_attn(const Params& prm, int grid, int hd, const void* q, const void* k, const void* v,
+static int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 148;
+  return n > 0 ? n : 148;
+}
+
+// `tiles` is the number of tile pairs (or an upper bound); the persistent
+// grid has one CTA per SM at most.
+static moga_status dispatch_attn(const Params& prm, int tiles, int hd, const void* q, const void* k, const void* v,
                                  cudaStream_t s) {
+  const int grid = std::min(tiles, sm_count());
   return hd == 128 ? launch_attn<128>(prm, grid, q, k, v, s) : launch_attn<64>(prm, grid, q, k, v, s);
 }
 
@@ -840,9 +933,9 @@ extern "C" moga_status moga_group_attn(const void* q, const void* k, const void*
   if ((st = launch_gather(prm, hd, q, k, v, ws, s)) != MOGA_OK) return st;
   const uint8_t* w = static_cast<const uint8_t*>(ws);
   const size_t bytes = (size_t)N * H * hd * 2;
-  // upper bound on the CTA count: sum_i ceil(n_i / 256) <= N / 256 + M
-  const int grid = (ceil_div((int)N, 2 * BM) + M) * H;
-  return dispatch_attn(prm, grid, hd, w, w + bytes, w + 2 * bytes, s);
+  // upper bound on the tile count: sum_i ceil(n_i / 256) <= N / 256 + M
+  const int tiles = (ceil_div((int)N, 2 * BM) + M) * H;
+  return dispatch_attn(prm, tiles, hd, w, w + bytes, w + 2 * bytes, s);
 }
 
 extern "C" moga_status stga_attn(const void* q, const void* k, const void* v, int32_t H, int32_t hd,

@@ -37,21 +37,29 @@ __global__ void mean3_tail_kernel(const float* __restrict__ acc, __nv_bfloat16* 
   if (i < n) out[i] = __float2bfloat16_rn(acc[i] / 3.0f);
 }
 
-// One warp: fixed-order fp64 reduction of the route partials.
-__global__ void balance_loss_kernel(const int32_t* __restrict__ counts, const float* __restrict__ partial,
-                                    int blocks, int N, int M, float alpha, double* __restrict__ loss) {
-  const int lane = threadIdx.x;
-  double fp = 0.0;
-  if (lane < M) {
-    double s = 0.0;
-    for (int b = 0; b < blocks; ++b) s += (double)partial[(size_t)b * M + lane];
-    const double F = (double)counts[lane] / (double)N;
-    const double P = s / (double)N;
-    fp = F * P;
-  }
+// One block of 8 warps: warp w sums the route partials of blocks w, w+8, ...
+// in fp64 (lane = group), then the warps are combined in a fixed order.
+__global__ void __launch_bounds__(256)
+balance_loss_kernel(const int32_t* __restrict__ counts, const float* __restrict__ partial, int blocks, int N,
+                    int M, float alpha, double* __restrict__ loss) {
+  __shared__ double part[8][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  double s = 0.0;
+  if (lane < M)
+    for (int b = warp; b < blocks; b += 8) s += (double)partial[(size_t)b * M + lane];
+  part[warp][lane] = s;
+  __syncthreads();
+  if (warp == 0) {
+    double fp = 0.0;
+    if (lane < M) {
+      double tot = 0.0;
+      for (int w = 0; w < 8; ++w) tot += part[w][lane];
+      fp = ((double)counts[lane] / (double)N) * (tot / (double)N);
+    }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) fp += __shfl_xor_sync(0xffffffffu, fp, off);
-  if (lane == 0) *loss = (double)alpha * (double)M * fp;
+    for (int off = 16; off > 0; off >>= 1) fp += __shfl_xor_sync(0xffffffffu, fp, off);
+    if (lane == 0) *loss = (double)alpha * (double)M * fp;
+  }
 }
 
 }  // namespace mean_detail
@@ -92,7 +100,7 @@ extern "C" moga_status moga_balance_loss(const int32_t* counts, const void* rout
   if (!counts || !route_ws || !loss) return fail(MOGA_ERR_INVALID_ARG, "moga_balance_loss: null pointer");
   if (N <= 0 || N > INT32_MAX) return fail(MOGA_ERR_INVALID_ARG, "moga_balance_loss: N=%lld out of range", (long long)N);
   if (M < 1 || M > 32) return fail(MOGA_ERR_INVALID_ARG, "moga_balance_loss: M=%d not in [1, 32]", M);
-  mean_detail::balance_loss_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+  mean_detail::balance_loss_kernel<<<1, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       counts, static_cast<const float*>(route_ws), route_blocks(N), (int)N, M, alpha, loss);
   return check_launch("moga_balance_loss");
 }

@@ -6,38 +6,53 @@
 // group; the blog (xugj520.cn) section 2.3 sketches the same bias-free layer.
 //
 // Design (HBM-bound: one read of x):
-//   * one thread per token, 128 tokens per block (4 warps);
-//   * x is read in 16-byte vectors through the read-only path; the 32 rows
-//     of a warp are disjoint so each 32-byte sector is fetched once and its
-//     second half is served from L1 on the next vector;
-//   * W_r is staged in shared memory as fp32 in chunks of KC rows of d,
-//     laid out [k][MP] (MP = M rounded up to 4) so one broadcast 128-bit
-//     load gives four groups' weights to the whole warp;
-//   * logits accumulate in fp32 registers (MP <= 32 accumulators).
+//   * four threads per token, 64 tokens per 256-thread block; thread s of a
+//     token reads the 16-byte chunks s, s+4, s+8, ... of the row, so the
+//     four threads of a token read 64 contiguous bytes per step and a warp
+//     reads 8 such segments (every 32-byte sector fully used);
+//   * several chunks are loaded before they are used, keeping enough bytes
+//     in flight per SM to cover HBM latency;
+//   * W_r is staged in shared memory as fp32 transposed to [M][k], so the
+//     four threads of a token read adjacent 32-byte pieces (no bank
+//     conflicts) and the 8 tokens of a warp share them (broadcast);
+//     d is processed in chunks that fit the shared-memory budget;
+//   * logits accumulate in fp32 registers, the four partial sums of a token
+//     are combined with two shuffles.
 #include "common.cuh"
 
 namespace moga {
 namespace route_detail {
 
-constexpr int kThreads = 128;      // tokens per block
-constexpr int kChunkBytes = 40 * 1024;
+constexpr int kThreads = 256;
+constexpr int kSub = 4;                       // threads per token
+constexpr int kTokens = kThreads / kSub;      // tokens per block
+constexpr int kSmemBudget = 64 * 1024;        // fp32 W_r chunk
+constexpr int kUnroll = 4;                    // 16-byte chunks loaded ahead per thread
 
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float* f) {
-  uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+template <typename T>
+struct Vec;
+template <>
+struct Vec<__nv_bfloat16> {
+  // 8 elements = 16 bytes
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float* f) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
   }
-}
-
-__device__ __forceinline__ void load8(const float* p, float* f) {
-  float4 a = __ldg(reinterpret_cast<const float4*>(p));
-  float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-}
+};
+template <>
+struct Vec<float> {
+  static __device__ __forceinline__ void load(const float* p, float* f) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  }
+};
 
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
 __device__ __forceinline__ float to_f32(float v) { return v; }
@@ -49,11 +64,12 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
              int32_t* __restrict__ group_id, float* __restrict__ gate_prob,
              float* __restrict__ psum_partial) {
   extern __shared__ float4 smem_f4[];
-  float* ws = reinterpret_cast<float*>(smem_f4);   // [KC][MP]
+  float* ws = reinterpret_cast<float*>(smem_f4);   // [MP][KC]
   __shared__ float red[kThreads / 32][MP];
 
   const int tid = threadIdx.x;
-  const int tok = blockIdx.x * kThreads + tid;
+  const int sub = tid & (kSub - 1);
+  const int tok = blockIdx.x * kTokens + tid / kSub;
   const bool active = tok < N;
   const T* xrow = x + (size_t)(active ? tok : 0) * d;
 
@@ -64,33 +80,60 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
   for (int k0 = 0; k0 < d; k0 += KC) {
     const int kc = min(KC, d - k0);
     __syncthreads();
-    for (int i = tid; i < kc * MP; i += kThreads) {
-      const int kk = i / MP, m = i % MP;
-      ws[i] = (m < M) ? to_f32(w_r[(size_t)(k0 + kk) * M + m]) : 0.f;
+    // one row of W_r (M contiguous values) per thread per step; all loads of
+    // a row are issued before the shared-memory stores
+    for (int kk = tid; kk < kc; kk += kThreads) {
+      const T* src = w_r + (size_t)(k0 + kk) * M;
+      float wv[MP];
+#pragma unroll
+      for (int m = 0; m < MP; ++m) wv[m] = (m < M) ? to_f32(__ldg(src + m)) : 0.f;
+#pragma unroll
+      for (int m = 0; m < MP; ++m) ws[m * KC + kk] = wv[m];
     }
     __syncthreads();
     if (active) {
-      for (int kk = 0; kk < kc; kk += 8) {
-        float xv[8];
-        load8(xrow + k0 + kk, xv);
+      const int nchunk = kc / 8;   // 8-element chunks in this part of the row
+      for (int c0 = sub; c0 < nchunk; c0 += kSub * kUnroll) {
+        float xv[kUnroll][8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float4* wv = reinterpret_cast<const float4*>(ws + (kk + e) * MP);
+        for (int u = 0; u < kUnroll; ++u) {
+          const int c = c0 + u * kSub;
+          if (c < nchunk) Vec<T>::load(xrow + k0 + 8 * c, xv[u]);
+        }
 #pragma unroll
-          for (int m4 = 0; m4 < MP / 4; ++m4) {
-            const float4 w4 = wv[m4];
-            acc[4 * m4 + 0] = fmaf(xv[e], w4.x, acc[4 * m4 + 0]);
-            acc[4 * m4 + 1] = fmaf(xv[e], w4.y, acc[4 * m4 + 1]);
-            acc[4 * m4 + 2] = fmaf(xv[e], w4.z, acc[4 * m4 + 2]);
-            acc[4 * m4 + 3] = fmaf(xv[e], w4.w, acc[4 * m4 + 3]);
+        for (int u = 0; u < kUnroll; ++u) {
+          const int c = c0 + u * kSub;
+          if (c < nchunk) {
+#pragma unroll
+            for (int m = 0; m < MP; ++m) {
+              const float4* wv = reinterpret_cast<const float4*>(ws + m * KC + 8 * c);
+              const float4 a = wv[0], b = wv[1];
+              float s = acc[m];
+              s = fmaf(xv[u][0], a.x, s);
+              s = fmaf(xv[u][1], a.y, s);
+              s = fmaf(xv[u][2], a.z, s);
+              s = fmaf(xv[u][3], a.w, s);
+              s = fmaf(xv[u][4], b.x, s);
+              s = fmaf(xv[u][5], b.y, s);
+              s = fmaf(xv[u][6], b.z, s);
+              s = fmaf(xv[u][7], b.w, s);
+              acc[m] = s;
+            }
           }
         }
       }
     }
   }
+  // combine the four partial logits of each token
+#pragma unroll
+  for (int m = 0; m < MP; ++m) {
+    acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], 1);
+    acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], 2);
+  }
 
   // softmax, argmax (lowest index wins a tie), gate
   float p[MP];
+  const bool writer = active && sub == 0;
   if (active) {
     float best = -INFINITY;
     int g = 0;
@@ -110,15 +153,17 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
     }
     const float inv = 1.f / z;
 #pragma unroll
-    for (int m = 0; m < MP; ++m) p[m] *= inv;
-    group_id[tok] = g;
-    gate_prob[tok] = 1.f / z;   // exp(r_g - max) = 1
+    for (int m = 0; m < MP; ++m) p[m] = writer ? p[m] * inv : 0.f;
+    if (writer) {
+      group_id[tok] = g;
+      gate_prob[tok] = inv;   // exp(r_g - max) = 1
+    }
   } else {
 #pragma unroll
     for (int m = 0; m < MP; ++m) p[m] = 0.f;
   }
 
-  // fixed-order block reduction of p(i|x): warp butterfly, then warps 0..3
+  // fixed-order block reduction of p(i|x): warp butterfly, then warps in order
   const int lane = tid & 31, warp = tid >> 5;
 #pragma unroll
   for (int m = 0; m < MP; ++m) {
@@ -139,11 +184,13 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
 template <typename T, int MP>
 moga_status launch(const void* x, const void* w_r, const float* bias, int N, int d, int M,
                    int32_t* g, float* gate, float* partial, cudaStream_t s) {
-  int KC = kChunkBytes / (MP * 4);
-  KC = (KC / 8) * 8;
-  if (KC > d) KC = d;
+  int KC = kSmemBudget / (MP * 4);
+  KC = (KC / 32) * 32;            // whole 8-element chunks for all four threads
+  if (KC >= d) KC = d;
   const size_t smem = (size_t)KC * MP * sizeof(float);
-  const int blocks = ceil_div(N, kThreads);
+  cudaError_t e = cudaFuncSetAttribute(route_kernel<T, MP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return fail(MOGA_ERR_CUDA, "moga_route: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+  const int blocks = ceil_div(N, kTokens);
   route_kernel<T, MP><<<blocks, kThreads, smem, s>>>(static_cast<const T*>(x), static_cast<const T*>(w_r),
                                                      bias, N, d, M, KC, g, gate, partial);
   return check_launch("moga_route");
@@ -166,7 +213,7 @@ moga_status dispatch(const void* x, const void* w_r, const float* bias, int N, i
 
 }  // namespace route_detail
 
-int route_blocks(int64_t N) { return ceil_div((int)N, route_detail::kThreads); }
+int route_blocks(int64_t N) { return ceil_div((int)N, route_detail::kTokens); }
 
 }  // namespace moga
 
