@@ -5,6 +5,7 @@ Usage: python -m sparse_attention_long_moga_b200.build
 from __future__ import annotations
 
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -40,12 +41,41 @@ def stale() -> bool:
     return any(os.path.getmtime(s) > t for s in srcs if os.path.exists(s))
 
 
+# The attention kernel launches at this many registers per thread and then
+# splits them between its warpgroups with setmaxnreg (csrc/attention.cu:
+# kLaunchRegs).  A different launch count would make the split unbalanced,
+# so the build refuses to produce such a library.
+ATTN_LAUNCH_REGS = 168
+
+
+def check_register_split(ptxas_log: str) -> None:
+    lines = ptxas_log.splitlines()
+    found = 0
+    for i, line in enumerate(lines):
+        if "Compiling entry function" in line and "attn_kernel" in line:
+            for nxt in lines[i + 1:i + 4]:
+                m = re.search(r"Used (\d+) registers", nxt)
+                if m:
+                    found += 1
+                    if int(m.group(1)) != ATTN_LAUNCH_REGS:
+                        raise RuntimeError("attention kernel compiled to %s registers per thread, expected %d "
+                                           "(the setmaxnreg split would not balance)" % (m.group(1), ATTN_LAUNCH_REGS))
+                    break
+    if found == 0:
+        raise RuntimeError("could not find the attention kernel's register count in the ptxas report")
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not stale():
         return LIB
     tmp = LIB + ".tmp"
-    cmd = [nvcc()] + flags(verbose) + ["-o", tmp] + [os.path.join(CSRC, s) for s in SOURCES]
-    subprocess.run(cmd, check=True)
+    cmd = [nvcc()] + flags(True) + ["-o", tmp] + [os.path.join(CSRC, s) for s in SOURCES]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if verbose or res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+    if res.returncode != 0:
+        raise subprocess.CalledProcessError(res.returncode, cmd, res.stdout, res.stderr)
+    check_register_split(res.stdout + res.stderr)
     os.replace(tmp, LIB)
     return LIB
 

@@ -19,6 +19,7 @@
 //     warp 8           producer: 3-D tiled TMA loads (128B swizzle) of the
 //                      two Q tiles and a 2-stage ring of K and V tiles
 //     warp 9           TMEM allocator; lane 0 issues tcgen05.mma
+//     warps 10-11      idle (complete the third warpgroup)
 //   TMEM columns: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
 //   The softmax writes P as bf16 pairs over the first 64 columns of its S
 //   and the P.V product reads it from there (A operand in tensor memory).
@@ -30,6 +31,7 @@
 // Every wait is bounded; on a timeout the CTA records MOGA_ERR_TIMEOUT,
 // drains what it has in flight, frees TMEM and exits.
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -43,7 +45,14 @@ namespace attn {
 
 constexpr int BM = 128;        // query rows per tile (two tiles per CTA)
 constexpr int BN = 128;        // key/value rows per tile
-constexpr int kThreads = 320;  // 10 warps
+constexpr int kThreads = 384;  // 12 warps: two softmax warpgroups + producer, MMA and two idle warps
+// Register split (setmaxnreg): the kernel launches at 168 registers per
+// thread (384 x 168 = 64512); the producer/MMA warpgroup gives back down to
+// 56 and the two softmax warpgroups take 224: 128 x 56 + 256 x 224 = 64512.
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 192;
+constexpr int kControlRegs = 120;
+static_assert(kThreads * kLaunchRegs == 128 * kControlRegs + 256 * kSoftmaxRegs, "register split must balance");
 constexpr int kMaxTG = 256;    // temporal groups per launch
 constexpr uint32_t kTmemCols = 512;
 constexpr int kHalfBytes = BM * 128;   // one 64-column half of a 128-row tile (16 KB)
@@ -246,6 +255,41 @@ __device__ __forceinline__ float poly_exp2(float x) {
   const float f = x - (t - 12582912.0f);
   const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Two exponentials with one SFU op: the pair of exponents is rounded to
+// f16x2 and ex2.approx.f16x2 returns both powers of two.  The inputs are
+// <= 8 (the reference max trails the true max by at most 2^8), so f16
+// keeps them to within 2^-7 absolute (within 2^-10 relative to the result
+// for the exponents near 0 that carry the softmax mass); the results are
+// rounded to bf16 for the P.V product anyway.
+#ifndef MOGA_SOFTMAX_X2
+#define MOGA_SOFTMAX_X2 1
+#endif
+#ifndef MOGA_P_TRUNC
+#define MOGA_P_TRUNC 0
+#endif
+#ifndef MOGA_EXP2_F16X2
+#define MOGA_EXP2_F16X2 0
+#endif
+__device__ __forceinline__ void exp2_pair(float xa, float xb, float& ea, float& eb) {
+#if MOGA_EXP2_F16X2
+  uint32_t h, e;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(xb), "f"(xa));   // xa -> low half
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(h));
+  __half2 r = *reinterpret_cast<__half2*>(&e);
+  ea = __low2float(r);
+  eb = __high2float(r);
+#else
+  ea = fast_exp2(xa);
+  eb = fast_exp2(xb);
+#endif
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -500,6 +544,10 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
   const uint32_t tmem = *tmem_slot;
   const long long timeout = p.timeout_cycles;
 
+  // Each warpgroup adjusts its register budget once, inside its own branch,
+  // so the code of each role is compiled against its own budget.
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
   if (warp == 8) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
@@ -632,7 +680,9 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
       mbar_drain(bar(B_MMA_END), 0, timeout);
     }
     __syncwarp();
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     // ---------------------------------------------------------------- softmax
     const int qt = warp >> 2;                            // query tile of this warpgroup
     const int row = (warp & 3) * 32 + lane;              // TMEM lane == query row
@@ -652,7 +702,14 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
         ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + qt), sc & 1, abort_flag, timeout));
         if (!ok) break;
         tc_fence_after();
+#if MOGA_SOFTMAX_X2
+        // scores as pairs, so the scale-and-shift and the row sum run as
+        // packed f32x2 operations (half the instructions)
+        float2 s2[BN / 2];
+        float* s = reinterpret_cast<float*>(s2);
+#else
         float s[BN];
+#endif
 #pragma unroll
         for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(s_addr + cc * 32, s + cc * 32);
         tmem_wait_ld();
@@ -662,17 +719,15 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
           for (int cc = 0; cc < BN; ++cc)
             if (cc >= valid) s[cc] = -INFINITY;
         }
-        // row max with 8 independent chains (a single chain would expose the
-        // max latency 127 times)
+        // row max with 8 independent chains of three-input max
         float mp[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mp[e] = s[e];
 #pragma unroll
-        for (int cc = 8; cc < BN; cc += 8)
+        for (int cc = 8; cc < BN; cc += 16)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) mp[e] = fmaxf(mp[e], s[cc + e]);
-        const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                               fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+          for (int e = 0; e < 8; ++e) mp[e] = max3(mp[e], s[cc + e], s[cc + 8 + e]);
+        const float mx = max3(max3(mp[0], mp[1], mp[2]), max3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
         const float m_new = fmaxf(m_run, mx * sl);
         // Move the reference max only when it grows by more than 2^8 (tile 0
         // always sets it); rows that move it rescale O and l after P is written.
@@ -680,21 +735,59 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
         const float m_old = m_run;
         if (j == 0 || need) m_run = m_new;
         const float neg_m = -m_run;
+#if MOGA_SOFTMAX_X2
+        const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(neg_m, neg_m);
+        float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int cc = 0; cc < BN / 16; ++cc) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float2 xab = __ffma2_rn(s2[cc * 8 + e], sl2, nm2);
+            const float2 pab = make_float2(fast_exp2(xab.x), fast_exp2(xab.y));
+            acc2[e & 3] = __fadd2_rn(acc2[e & 3], pab);
+            pk[e] = pack_bf16x2(pab.x, pab.y);
+          }
+          // P overwrites S columns [8cc, 8cc+8), whose scores were read above
+          tmem_st8(s_addr + cc * 8, pk);
+        }
+        const float2 acc01 = __fadd2_rn(acc2[0], acc2[1]), acc23 = __fadd2_rn(acc2[2], acc2[3]);
+        const float row_sum = (acc01.x + acc01.y) + (acc23.x + acc23.y);
+#else
         float sp[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
 #pragma unroll
         for (int cc = 0; cc < BN / 16; ++cc) {
           uint32_t pk[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float a = fast_exp2(fmaf(s[cc * 16 + 2 * e], sl, neg_m));
+            const float xa = fmaf(s[cc * 16 + 2 * e], sl, neg_m);
             const float xb = fmaf(s[cc * 16 + 2 * e + 1], sl, neg_m);
-            const float b = (MOGA_POLY_EXP2 && (e & 1)) ? poly_exp2(xb) : fast_exp2(xb);
+            float a, b;
+            if (MOGA_POLY_EXP2 && (e & 1)) {
+              a = fast_exp2(xa);
+              b = poly_exp2(xb);
+            } else {
+              exp2_pair(xa, xb, a, b);
+            }
+#if MOGA_P_TRUNC
+            // P rounded toward zero to bf16 by keeping the high halves (an
+            // ALU byte permute instead of a conversion), and the row sum taken
+            // over the same truncated values, so numerator and denominator of
+            // the softmax use identical weights
+            const uint32_t ua = __float_as_uint(a) & 0xFFFF0000u;
+            const uint32_t ub = __float_as_uint(b) & 0xFFFF0000u;
+            sp[e & 3] += __uint_as_float(ua) + __uint_as_float(ub);
+            pk[e] = __byte_perm(ua, ub, 0x7632);
+#else
             sp[e & 3] += a + b;
             pk[e] = pack_bf16x2(a, b);
+#endif
           }
           // P overwrites S columns [8cc, 8cc+8), whose scores were read above
           tmem_st8(s_addr + cc * 8, pk);
         }
+        const float row_sum = (sp[0] + sp[1]) + (sp[2] + sp[3]);
+#endif
         if (__any_sync(0xffffffffu, need)) {
           // P.V of tile j-1 finished before S of tile j (issue order), so O
           // may be rescaled here, before P_j is released to the MMA warp
@@ -710,7 +803,7 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
           }
           l_run *= f;
         }
-        l_run += (sp[0] + sp[1]) + (sp[2] + sp[3]);
+        l_run += row_sum;
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(B_P_FULL + qt));

@@ -64,7 +64,7 @@ balance_loss_kernel(const int32_t* __restrict__ counts, const float* __restrict_
 
 }  // namespace mean_detail
 
-int route_blocks(int64_t N);
+int route_blocks(int64_t N, int M);
 
 }  // namespace moga
 
@@ -101,6 +101,6 @@ extern "C" moga_status moga_balance_loss(const int32_t* counts, const void* rout
   if (N <= 0 || N > INT32_MAX) return fail(MOGA_ERR_INVALID_ARG, "moga_balance_loss: N=%lld out of range", (long long)N);
   if (M < 1 || M > 32) return fail(MOGA_ERR_INVALID_ARG, "moga_balance_loss: M=%d not in [1, 32]", M);
   mean_detail::balance_loss_kernel<<<1, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      counts, static_cast<const float*>(route_ws), route_blocks(N), (int)N, M, alpha, loss);
+      counts, static_cast<const float*>(route_ws), route_blocks(N, M), (int)N, M, alpha, loss);
   return check_launch("moga_balance_loss");
 }

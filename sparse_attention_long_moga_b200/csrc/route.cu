@@ -6,10 +6,11 @@
 // group; the blog (xugj520.cn) section 2.3 sketches the same bias-free layer.
 //
 // Design (HBM-bound: one read of x):
-//   * four threads per token, 64 tokens per 256-thread block; thread s of a
-//     token reads the 16-byte chunks s, s+4, s+8, ... of the row, so the
-//     four threads of a token read 64 contiguous bytes per step and a warp
-//     reads 8 such segments (every 32-byte sector fully used);
+//   * four threads per token; thread s of a token reads the 16-byte chunks
+//     s, s+4, s+8, ... of the row, so the four threads of a token read 64
+//     contiguous bytes per step and a warp reads 8 such segments (every
+//     32-byte sector fully used); each thread serves up to 4 tokens so that
+//     each shared-memory read of W_r feeds several tokens;
 //   * several chunks are loaded before they are used, keeping enough bytes
 //     in flight per SM to cover HBM latency;
 //   * W_r is staged in shared memory as fp32 transposed to [M][k], so the
@@ -57,25 +58,41 @@ struct Vec<float> {
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
 __device__ __forceinline__ float to_f32(float v) { return v; }
 
+// TT tokens per thread (strided by kTokens inside the block): every W_r value
+// read from shared memory feeds TT tokens, which keeps the shared-memory
+// traffic per byte of x below the HBM rate.
+template <int MP>
+struct Tokens {
+  static constexpr int value = MP <= 8 ? 4 : (MP <= 16 ? 2 : 1);
+};
+
 template <typename T, int MP>
 __global__ void __launch_bounds__(kThreads)
 route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __restrict__ bias,
              int N, int d, int M, int KC,
              int32_t* __restrict__ group_id, float* __restrict__ gate_prob,
              float* __restrict__ psum_partial) {
+  constexpr int TT = Tokens<MP>::value;
+  constexpr int U = 2;   // 16-byte chunks of each token loaded ahead
   extern __shared__ float4 smem_f4[];
   float* ws = reinterpret_cast<float*>(smem_f4);   // [MP][KC]
   __shared__ float red[kThreads / 32][MP];
 
   const int tid = threadIdx.x;
   const int sub = tid & (kSub - 1);
-  const int tok = blockIdx.x * kTokens + tid / kSub;
-  const bool active = tok < N;
-  const T* xrow = x + (size_t)(active ? tok : 0) * d;
-
-  float acc[MP];
+  const int tok0 = blockIdx.x * kTokens * TT + tid / kSub;
+  const T* xrow[TT];
 #pragma unroll
-  for (int m = 0; m < MP; ++m) acc[m] = 0.f;
+  for (int t = 0; t < TT; ++t) {
+    const int tok = tok0 + t * kTokens;
+    xrow[t] = x + (size_t)(tok < N ? tok : 0) * d;
+  }
+
+  float acc[TT][MP];
+#pragma unroll
+  for (int t = 0; t < TT; ++t)
+#pragma unroll
+    for (int m = 0; m < MP; ++m) acc[t][m] = 0.f;
 
   for (int k0 = 0; k0 < d; k0 += KC) {
     const int kc = min(KC, d - k0);
@@ -91,93 +108,94 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
       for (int m = 0; m < MP; ++m) ws[m * KC + kk] = wv[m];
     }
     __syncthreads();
-    if (active) {
-      const int nchunk = kc / 8;   // 8-element chunks in this part of the row
-      for (int c0 = sub; c0 < nchunk; c0 += kSub * kUnroll) {
-        float xv[kUnroll][8];
+    const int nchunk = kc / 8;   // 8-element chunks in this part of the row
+    for (int c0 = sub; c0 < nchunk; c0 += kSub * U) {
+      float xv[U][TT][8];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-          const int c = c0 + u * kSub;
-          if (c < nchunk) Vec<T>::load(xrow + k0 + 8 * c, xv[u]);
-        }
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + u * kSub;
+        if (c < nchunk)
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-          const int c = c0 + u * kSub;
-          if (c < nchunk) {
+          for (int t = 0; t < TT; ++t) Vec<T>::load(xrow[t] + k0 + 8 * c, xv[u][t]);
+      }
 #pragma unroll
-            for (int m = 0; m < MP; ++m) {
-              const float4* wv = reinterpret_cast<const float4*>(ws + m * KC + 8 * c);
-              const float4 a = wv[0], b = wv[1];
-              float s = acc[m];
-              s = fmaf(xv[u][0], a.x, s);
-              s = fmaf(xv[u][1], a.y, s);
-              s = fmaf(xv[u][2], a.z, s);
-              s = fmaf(xv[u][3], a.w, s);
-              s = fmaf(xv[u][4], b.x, s);
-              s = fmaf(xv[u][5], b.y, s);
-              s = fmaf(xv[u][6], b.z, s);
-              s = fmaf(xv[u][7], b.w, s);
-              acc[m] = s;
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + u * kSub;
+        if (c < nchunk) {
+#pragma unroll
+          for (int m = 0; m < MP; ++m) {
+            const float4* wv = reinterpret_cast<const float4*>(ws + m * KC + 8 * c);
+            const float4 a = wv[0], b = wv[1];
+#pragma unroll
+            for (int t = 0; t < TT; ++t) {
+              float sacc = acc[t][m];
+              sacc = fmaf(xv[u][t][0], a.x, sacc);
+              sacc = fmaf(xv[u][t][1], a.y, sacc);
+              sacc = fmaf(xv[u][t][2], a.z, sacc);
+              sacc = fmaf(xv[u][t][3], a.w, sacc);
+              sacc = fmaf(xv[u][t][4], b.x, sacc);
+              sacc = fmaf(xv[u][t][5], b.y, sacc);
+              sacc = fmaf(xv[u][t][6], b.z, sacc);
+              sacc = fmaf(xv[u][t][7], b.w, sacc);
+              acc[t][m] = sacc;
             }
           }
         }
       }
     }
   }
-  // combine the four partial logits of each token
-#pragma unroll
-  for (int m = 0; m < MP; ++m) {
-    acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], 1);
-    acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], 2);
-  }
 
-  // softmax, argmax (lowest index wins a tie), gate
-  float p[MP];
-  const bool writer = active && sub == 0;
-  if (active) {
-    float best = -INFINITY;
-    int g = 0;
+  float psum[MP];
+#pragma unroll
+  for (int m = 0; m < MP; ++m) psum[m] = 0.f;
+#pragma unroll
+  for (int t = 0; t < TT; ++t) {
+    const int tok = tok0 + t * kTokens;
+    // combine the four partial logits of the token
 #pragma unroll
     for (int m = 0; m < MP; ++m) {
-      if (m < M) {
-        const float r = acc[m] + (bias ? __ldg(bias + m) : 0.f);
-        acc[m] = r;
-        if (r > best) { best = r; g = m; }
+      acc[t][m] += __shfl_xor_sync(0xffffffffu, acc[t][m], 1);
+      acc[t][m] += __shfl_xor_sync(0xffffffffu, acc[t][m], 2);
+    }
+    if (tok < N && sub == 0) {
+      // softmax, argmax (lowest index wins a tie), gate
+      float best = -INFINITY;
+      int g = 0;
+      float r[MP];
+#pragma unroll
+      for (int m = 0; m < MP; ++m) {
+        r[m] = acc[t][m] + ((bias && m < M) ? __ldg(bias + m) : 0.f);
+        if (m < M && r[m] > best) { best = r[m]; g = m; }
       }
-    }
-    float z = 0.f;
+      float e[MP], z = 0.f;
 #pragma unroll
-    for (int m = 0; m < MP; ++m) {
-      p[m] = (m < M) ? expf(acc[m] - best) : 0.f;
-      z += p[m];
-    }
-    const float inv = 1.f / z;
+      for (int m = 0; m < MP; ++m) {
+        e[m] = (m < M) ? expf(r[m] - best) : 0.f;
+        z += e[m];
+      }
+      const float inv = 1.f / z;
 #pragma unroll
-    for (int m = 0; m < MP; ++m) p[m] = writer ? p[m] * inv : 0.f;
-    if (writer) {
+      for (int m = 0; m < MP; ++m) psum[m] += e[m] * inv;
       group_id[tok] = g;
       gate_prob[tok] = inv;   // exp(r_g - max) = 1
     }
-  } else {
-#pragma unroll
-    for (int m = 0; m < MP; ++m) p[m] = 0.f;
   }
 
   // fixed-order block reduction of p(i|x): warp butterfly, then warps in order
   const int lane = tid & 31, warp = tid >> 5;
 #pragma unroll
   for (int m = 0; m < MP; ++m) {
-    float v = p[m];
+    float v = psum[m];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
     if (lane == 0) red[warp][m] = v;
   }
   __syncthreads();
   if (tid < M) {
-    float s = 0.f;
+    float sacc = 0.f;
 #pragma unroll
-    for (int w = 0; w < kThreads / 32; ++w) s += red[w][tid];
-    psum_partial[(size_t)blockIdx.x * M + tid] = s;
+    for (int w = 0; w < kThreads / 32; ++w) sacc += red[w][tid];
+    psum_partial[(size_t)blockIdx.x * M + tid] = sacc;
   }
 }
 
@@ -190,7 +208,7 @@ moga_status launch(const void* x, const void* w_r, const float* bias, int N, int
   const size_t smem = (size_t)KC * MP * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(route_kernel<T, MP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return fail(MOGA_ERR_CUDA, "moga_route: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-  const int blocks = ceil_div(N, kTokens);
+  const int blocks = ceil_div(N, kTokens * Tokens<MP>::value);
   route_kernel<T, MP><<<blocks, kThreads, smem, s>>>(static_cast<const T*>(x), static_cast<const T*>(w_r),
                                                      bias, N, d, M, KC, g, gate, partial);
   return check_launch("moga_route");
@@ -213,13 +231,18 @@ moga_status dispatch(const void* x, const void* w_r, const float* bias, int N, i
 
 }  // namespace route_detail
 
-int route_blocks(int64_t N) { return ceil_div((int)N, route_detail::kTokens); }
+// Blocks of the route launch for (N, M): the Σp partials have one row per block.
+int route_blocks(int64_t N, int M) {
+  const int mp = (M + 3) / 4 * 4;
+  const int tt = mp <= 8 ? 4 : (mp <= 16 ? 2 : 1);
+  return ceil_div((int)N, route_detail::kTokens * tt);
+}
 
 }  // namespace moga
 
 extern "C" size_t moga_route_ws_bytes(int64_t N, int32_t M) {
   if (N <= 0 || N > INT32_MAX || M < 1 || M > 32) return 0;
-  return (size_t)moga::route_blocks(N) * (size_t)M * sizeof(float);
+  return (size_t)moga::route_blocks(N, M) * (size_t)M * sizeof(float);
 }
 
 extern "C" moga_status moga_route(const void* x, const void* w_r, moga_dtype dt, const float* bias,
