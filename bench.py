@@ -121,6 +121,21 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(local_ms: float, device=None) -> float:
+    """Job time: the largest per-rank device time (a one-element all-reduce outside the timed region)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, tokens_per_rank: int, steps: int, job_ms: float) -> float:
+    """Whole-job tokens/s: every rank runs its own sequence of `tokens_per_rank` tokens per step."""
+    return world * tokens_per_rank * steps / (job_ms / 1000.0)
+
+
 def make_inputs(wl):
     """Seeded synthetic inputs (stored margin redraws applied), as numpy stored values."""
     redraw = W.redraw_map(wl)
@@ -254,23 +269,31 @@ def run_ours(args):
     gs, keep = moga.geom_struct(geom)
     scale = 1.0 / math.sqrt(hd)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    ev_moga = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    CALLS = ("route", "permute", "moga_group_attn", "stga_attn", "visual_attn_mean", "moga_balance_loss")
+    evl = [torch.cuda.Event(enable_timing=True) for _ in range(len(CALLS) + 1)]
 
-    def step(xd, qd, kd, vd, time_moga=False):
+    def step(xd, qd, kd, vd, timed=False):
         c = moga.check
+
+        def mark(i):
+            if timed:
+                evl[i].record(stream)
+        mark(0)
         c(L.moga_route(P(xd), P(w_r), moga.MOGA_BF16, None, N, wl.d, M, P(g), P(gate), P(rws), rws.numel(), sp),
           "route")
+        mark(1)
         c(L.moga_permute(P(g), N, M, P(perm), P(cu), P(counts), P(mx), P(pws), pws.numel(), sp), "permute")
-        if time_moga:
-            ev_moga[0].record(stream)
-        c(L.moga_group_attn(P(qd), P(kd), P(vd), N, H, hd, P(perm), P(cu), M, P(gate), scale, P(o_acc), P(aws), aws.numel(), sp),
-          "moga")
-        if time_moga:
-            ev_moga[1].record(stream)
+        mark(2)
+        c(L.moga_group_attn(P(qd), P(kd), P(vd), N, H, hd, P(perm), P(cu), M, P(gate), scale, P(o_acc), P(aws),
+                            aws.numel(), sp), "moga")
+        mark(3)
         c(L.stga_attn(P(qd), P(kd), P(vd), H, hd, moga.ctypes.byref(gs), scale, P(o_acc), P(aws), aws.numel(),
-                        sp), "stga")
+                      sp), "stga")
+        mark(4)
         c(L.visual_attn_mean(P(o_acc), o_acc.numel(), P(out), sp), "mean")
+        mark(5)
         c(L.moga_balance_loss(P(counts), P(rws), N, M, wl.alpha, P(loss), sp), "loss")
+        mark(6)
 
     # route 1, permute 3, MoGA gather + attention 2, STGA gather + window + frame 3, mean 1 (+tail), loss 1
     launches_per_step = 1 + 3 + 2 + 3 + 1 + 1 + (1 if (N * H * hd) % 8 else 0)
@@ -283,7 +306,7 @@ def run_ours(args):
     # ---- device-timed region: K steps, L2 flushed between steps
     sampler = ClockSampler(local)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    moga_ms = []
+    call_ms = {name: [] for name in CALLS}
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -291,20 +314,20 @@ def run_ours(args):
     for i in range(args.steps):
         flush.zero_()
         evs[i][0].record(stream)
-        step(x, q, k, v, time_moga=True)
+        step(x, q, k, v, timed=True)
         evs[i][1].record(stream)
-        ev_moga[1].synchronize()
-        moga_ms.append(ev_moga[0].elapsed_time(ev_moga[1]))
+        evl[-1].synchronize()
+        for j, name in enumerate(CALLS):
+            call_ms[name].append(evl[j].elapsed_time(evl[j + 1]))
+    moga_ms = call_ms["moga_group_attn"]
     torch.cuda.synchronize()
     clocks = sampler.stop()
     moga.device_status()
     dev_ms = sum(a.elapsed_time(b) for a, b in evs)
-    t = torch.tensor([dev_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.barrier()
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    job_ms = float(t.item())
-    value = world * N * args.steps / (job_ms / 1000.0)
+    job_ms = max_over_ranks(dev_ms, dev)
+    value = job_throughput(world, N, args.steps, job_ms)
 
     # ---- end to end through the public API: pinned host inputs in, result out
     hx, hq, hk, hv = (torch.from_numpy(inp[n].view(np.int16)).pin_memory() for n in ("x", "q", "k", "v"))
@@ -328,10 +351,7 @@ def run_ours(args):
         e_evs[i][1].record(stream)
     torch.cuda.synchronize()
     e2e_ms = sum(a.elapsed_time(b) for a, b in e_evs)
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = world * N * args.steps / (float(te.item()) / 1000.0)
+    e2e_value = job_throughput(world, N, args.steps, max_over_ranks(e2e_ms, dev))
 
     counts_h = counts.cpu().numpy()
     fl_moga = moga_flops(counts_h, H, hd)
@@ -344,11 +364,15 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": job_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded counter-based generator; no dataset)",
         "config": config_dict(wl),
-        "roofline": {"bound": "tensor", "kernel": "group_attn_kernel<128> (MoGA groups)", "achieved": achieved,
+        "roofline": {"bound": "tensor",
+                     "kernel": "moga_group_attn call = gather3_kernel (segment-order copy) + attn_kernel<128>",
+                     "achieved": achieved,
                      "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
                      "peak_kind": "%s burst dense bf16" % pk_kind, "traffic": None,
                      "flops_per_launch": fl_moga, "launch_ms": moga_avg_s * 1e3},
         "layer_tflops": (fl_moga + fl_stga) / (job_ms / args.steps / 1000.0) / 1e12,
+        "breakdown_ms": {name: statistics.median(v) for name, v in call_ms.items()},
+        "stga_tflops": fl_stga / (statistics.median(call_ms["stga_attn"]) / 1000.0) / 1e12,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,

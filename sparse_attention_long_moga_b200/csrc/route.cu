@@ -6,26 +6,26 @@
 // group; the blog (xugj520.cn) section 2.3 sketches the same bias-free layer.
 //
 // Design (HBM-bound: one read of x):
-//   * four threads per token; thread s of a token reads the 16-byte chunks
-//     s, s+4, s+8, ... of the row, so the four threads of a token read 64
-//     contiguous bytes per step and a warp reads 8 such segments (every
-//     32-byte sector fully used); each thread serves up to 4 tokens so that
-//     each shared-memory read of W_r feeds several tokens;
+//   * eight threads per token; thread s of a token reads the 16-byte chunks
+//     s, s+8, s+16, ... of the row, so the eight threads of a token read 128
+//     contiguous bytes per step (every sector fully used); each thread
+//     serves up to 4 tokens so that each shared-memory read of W_r feeds
+//     several tokens;
 //   * several chunks are loaded before they are used, keeping enough bytes
 //     in flight per SM to cover HBM latency;
 //   * W_r is staged in shared memory as fp32 transposed to [M][k], so the
-//     four threads of a token read adjacent 32-byte pieces (no bank
-//     conflicts) and the 8 tokens of a warp share them (broadcast);
+//     eight threads of a token read adjacent 32-byte pieces and the 4 tokens
+//     of a warp share them (broadcast);
 //     d is processed in chunks that fit the shared-memory budget;
-//   * logits accumulate in fp32 registers, the four partial sums of a token
-//     are combined with two shuffles.
+//   * logits accumulate in fp32 registers, the eight partial sums of a token
+//     are combined with three shuffles.
 #include "common.cuh"
 
 namespace moga {
 namespace route_detail {
 
 constexpr int kThreads = 256;
-constexpr int kSub = 4;                       // threads per token
+constexpr int kSub = 8;                       // threads per token
 constexpr int kTokens = kThreads / kSub;      // tokens per block
 constexpr int kSmemBudget = 64 * 1024;        // fp32 W_r chunk
 constexpr int kUnroll = 4;                    // 16-byte chunks loaded ahead per thread
@@ -63,7 +63,7 @@ __device__ __forceinline__ float to_f32(float v) { return v; }
 // traffic per byte of x below the HBM rate.
 template <int MP>
 struct Tokens {
-  static constexpr int value = MP <= 8 ? 4 : (MP <= 16 ? 2 : 1);
+  static constexpr int value = MP <= 8 ? 4 : 2;
 };
 
 template <typename T, int MP>
@@ -151,11 +151,12 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
 #pragma unroll
   for (int t = 0; t < TT; ++t) {
     const int tok = tok0 + t * kTokens;
-    // combine the four partial logits of the token
+    // combine the eight partial logits of the token
 #pragma unroll
     for (int m = 0; m < MP; ++m) {
       acc[t][m] += __shfl_xor_sync(0xffffffffu, acc[t][m], 1);
       acc[t][m] += __shfl_xor_sync(0xffffffffu, acc[t][m], 2);
+      acc[t][m] += __shfl_xor_sync(0xffffffffu, acc[t][m], 4);
     }
     if (tok < N && sub == 0) {
       // softmax, argmax (lowest index wins a tie), gate
@@ -203,7 +204,7 @@ template <typename T, int MP>
 moga_status launch(const void* x, const void* w_r, const float* bias, int N, int d, int M,
                    int32_t* g, float* gate, float* partial, cudaStream_t s) {
   int KC = kSmemBudget / (MP * 4);
-  KC = (KC / 32) * 32;            // whole 8-element chunks for all four threads
+  KC = (KC / (8 * kSub)) * (8 * kSub);   // whole 8-element chunks for every thread of a token
   if (KC >= d) KC = d;
   const size_t smem = (size_t)KC * MP * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(route_kernel<T, MP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -234,7 +235,7 @@ moga_status dispatch(const void* x, const void* w_r, const float* bias, int N, i
 // Blocks of the route launch for (N, M): the Σp partials have one row per block.
 int route_blocks(int64_t N, int M) {
   const int mp = (M + 3) / 4 * 4;
-  const int tt = mp <= 8 ? 4 : (mp <= 16 ? 2 : 1);
+  const int tt = mp <= 8 ? 4 : 2;
   return ceil_div((int)N, route_detail::kTokens * tt);
 }
 

@@ -161,14 +161,28 @@ def _round_like(wl: Workload, a: np.ndarray) -> np.ndarray:
     return bf16_bits_to_f64(to_bf16_bits(a))
 
 
+def _parallel_chunks(n: int, chunk: int, fn) -> None:
+    """Run fn(start, stop) over [0, n) in chunks on a thread pool (numpy releases the GIL)."""
+    starts = list(range(0, n, chunk))
+    if len(starts) <= 2:
+        for s0 in starts:
+            fn(s0, min(s0 + chunk, n))
+        return
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+        list(ex.map(lambda s0: fn(s0, min(s0 + chunk, n)), starts))
+
+
 def x_stored(wl: Workload, redraw: dict | None = None, rows: np.ndarray | None = None,
              chunk: int = 8192) -> np.ndarray:
     """Router input in its stored form: float32 array or bf16 bits (uint16), [len(rows), d]."""
     rows = np.arange(wl.N) if rows is None else np.asarray(rows)
     out = np.empty((len(rows), wl.d), dtype=np.float32 if wl.x_dtype == "f32" else np.uint16)
-    for s in range(0, len(rows), chunk):
-        v = x_rows_f64(wl, rows[s:s + chunk], redraw)
-        out[s:s + chunk] = v.astype(np.float32) if wl.x_dtype == "f32" else to_bf16_bits(v)
+
+    def fill(a, b):
+        v = x_rows_f64(wl, rows[a:b], redraw)
+        out[a:b] = v.astype(np.float32) if wl.x_dtype == "f32" else to_bf16_bits(v)
+    _parallel_chunks(len(rows), chunk, fill)
     return out
 
 
@@ -218,9 +232,10 @@ def qkv_rows_bits(wl: Workload, which: str, rows: np.ndarray, redraw: dict | Non
 
 def qkv_stored(wl: Workload, which: str, redraw: dict | None = None, chunk: int = 4096) -> np.ndarray:
     out = np.empty((wl.N, wl.H, wl.hd), dtype=np.uint16)
-    for s in range(0, wl.N, chunk):
-        r = np.arange(s, min(s + chunk, wl.N))
-        out[s:s + len(r)] = qkv_rows_bits(wl, which, r, redraw)
+
+    def fill(a, b):
+        out[a:b] = qkv_rows_bits(wl, which, np.arange(a, b), redraw)
+    _parallel_chunks(wl.N, chunk, fill)
     return out
 
 

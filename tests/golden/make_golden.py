@@ -34,11 +34,13 @@ SKEW_TARGET = 0.40
 def route_probs(wl, rows, redraw, chunk=16384):
     w = W.w_r_f64(wl)
     b = W.bias_f64(wl)
-    out = []
-    for s in range(0, len(rows), chunk):
-        x = W.x_rows_f64(wl, rows[s:s + chunk], redraw)
-        out.append(route.probabilities(route.logits(x, w, b)))
-    return np.concatenate(out)
+    out = np.empty((len(rows), wl.M))
+
+    def fill(a, z):
+        x = W.x_rows_f64(wl, rows[a:z], redraw)
+        out[a:z] = route.probabilities(route.logits(x, w, b))
+    W._parallel_chunks(len(rows), chunk, fill)
+    return out
 
 
 def find_skew_bias(wl):

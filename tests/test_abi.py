@@ -40,7 +40,7 @@ def test_every_declared_symbol_is_exported(lib):
 def test_workspace_sizes(lib):
     assert lib.moga_route_ws_bytes(0, 5) == 0
     assert lib.moga_route_ws_bytes(1000, 33) == 0
-    assert lib.moga_route_ws_bytes(32760, 5) == 128 * 5 * 4
+    assert lib.moga_route_ws_bytes(32760, 5) == 256 * 5 * 4
     assert lib.moga_permute_ws_bytes(32760, 5) == 2 * 16 * 5 * 4
     assert lib.moga_permute_ws_bytes(-1, 5) == 0
 
