@@ -256,7 +256,7 @@ def run_ours(args):
     # persistent buffers: the step allocates nothing
     g = torch.empty(N, dtype=torch.int32, device=dev)
     gate = torch.empty(N, dtype=torch.float32, device=dev)
-    rws = torch.empty(max(L.moga_route_ws_bytes(N, M), 16), dtype=torch.uint8, device=dev)
+    rws = torch.empty(max(L.moga_route_ws_bytes(N, wl.d, M), 16), dtype=torch.uint8, device=dev)
     pws = torch.empty(max(L.moga_permute_ws_bytes(N, M), 16), dtype=torch.uint8, device=dev)
     perm = torch.empty(N, dtype=torch.int32, device=dev)
     cu = torch.empty(M + 1, dtype=torch.int32, device=dev)
@@ -295,8 +295,9 @@ def run_ours(args):
         c(L.moga_balance_loss(P(counts), P(rws), N, M, wl.alpha, P(loss), sp), "loss")
         mark(6)
 
-    # route 1, permute 3, MoGA gather + attention 2, STGA gather + window + frame 3, mean 1 (+tail), loss 1
-    launches_per_step = 1 + 3 + 2 + 3 + 1 + 1 + (1 if (N * H * hd) % 8 else 0)
+    # route 2 (W_r^T copy + tensor-core router), permute 3, MoGA gather + attention 2,
+    # STGA gather + window + frame 3, mean 1 (+tail), loss 1
+    launches_per_step = 2 + 3 + 2 + 3 + 1 + 1 + (1 if (N * H * hd) % 8 else 0)
 
     for _ in range(args.warmup):
         flush.zero_()

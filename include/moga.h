@@ -75,11 +75,15 @@ typedef struct {
  * w_r:       [d][M], same dtype as x
  * bias:      [M] fp32 or NULL (the pages' router has no bias)
  * group_id:  [N] int32 out;  gate_prob: [N] fp32 out
- * ws:        workspace of at least moga_route_ws_bytes(N, M) bytes; on return
- *            it holds per-block partial sums of p(i|x) that
- *            moga_balance_loss() reads.  Keep it until the loss is taken.
+ * ws:        workspace of at least moga_route_ws_bytes(N, d, M) bytes, 256-byte
+ *            aligned; on return it holds partial sums of p(i|x) (one row of
+ *            M per 32 tokens) that moga_balance_loss() reads.  Keep it until the
+ *            loss is taken.  bf16 inputs run on the tensor cores (x tiles
+ *            staged by TMA, fp32 accumulation in tensor memory); fp32 inputs
+ *            on the FMA pipe.
+ * moga_route_ws_bytes returns 0 for arguments moga_route would reject.
  */
-size_t moga_route_ws_bytes(int64_t N, int32_t M);
+size_t moga_route_ws_bytes(int64_t N, int32_t d, int32_t M);
 moga_status moga_route(const void* x, const void* w_r, moga_dtype dt, const float* bias,
                        int64_t N, int32_t d, int32_t M,
                        int32_t* group_id, float* gate_prob,

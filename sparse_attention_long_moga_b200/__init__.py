@@ -58,7 +58,7 @@ def moga_route(x: torch.Tensor, w_r: torch.Tensor, bias: torch.Tensor | None = N
     if bias is not None:
         _need(bias, torch.float32, "bias", 1)
     L = lib()
-    ws_bytes = L.moga_route_ws_bytes(N, M)
+    ws_bytes = L.moga_route_ws_bytes(N, d, M)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=x.device)
     g = torch.empty(N, dtype=torch.int32, device=x.device)
     gate = torch.empty(N, dtype=torch.float32, device=x.device)

@@ -21,7 +21,7 @@ MOGA_F32, MOGA_BF16 = 0, 1
 # exported symbol -> (restype, argtypes); the same list include/moga.h declares
 _P, _I32, _I64, _F32, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
-    "moga_route_ws_bytes": (_SZ, [_I64, _I32]),
+    "moga_route_ws_bytes": (_SZ, [_I64, _I32, _I32]),
     "moga_route": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _I64, _I32, _I32, _P, _P, _P, _SZ, _P]),
     "moga_permute_ws_bytes": (_SZ, [_I64, _I32]),
     "moga_permute": (ctypes.c_int, [_P, _I64, _I32, _P, _P, _P, _P, _P, _SZ, _P]),

@@ -37,34 +37,57 @@ __global__ void mean3_tail_kernel(const float* __restrict__ acc, __nv_bfloat16* 
   if (i < n) out[i] = __float2bfloat16_rn(acc[i] / 3.0f);
 }
 
-// One block of 8 warps: warp w sums the route partials of blocks w, w+8, ...
-// in fp64 (lane = group), then the warps are combined in a fixed order.
-__global__ void __launch_bounds__(256)
-balance_loss_kernel(const int32_t* __restrict__ counts, const float* __restrict__ partial, int blocks, int N,
+// One block of 1024 threads.  The partials form a [rows][M] fp32 array; with
+// S = M * floor(1024 / M), thread t < S sums the elements t, t + S, t + 2S, ...
+// (all of group t % M) in fp64; the per-thread sums are then folded per group
+// in a fixed order (32 strided slices, then the 32 slice sums), so the result
+// does not depend on scheduling.
+__global__ void __launch_bounds__(1024)
+balance_loss_kernel(const int32_t* __restrict__ counts, const float* __restrict__ partial, int rows, int N,
                     int M, float alpha, double* __restrict__ loss) {
-  __shared__ double part[8][32];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __shared__ double part[1024];
+  __shared__ double slice[32][32];
+  const int t = threadIdx.x;
+  const int R = 1024 / M;            // per-thread sums per group
+  const int S = R * M;
+  const int64_t n = (int64_t)rows * M;
   double s = 0.0;
-  if (lane < M)
-    for (int b = warp; b < blocks; b += 8) s += (double)partial[(size_t)b * M + lane];
-  part[warp][lane] = s;
+  if (t < S) {
+    double s1 = 0.0;
+    int64_t i = t;
+    for (; i + S < n; i += 2 * (int64_t)S) {
+      s += (double)partial[i];
+      s1 += (double)partial[i + S];
+    }
+    if (i < n) s += (double)partial[i];
+    s += s1;
+  }
+  part[t] = s;
   __syncthreads();
-  if (warp == 0) {
+  // slice j of group m: per-thread sums r = j, j + 32, ... (thread r * M + m)
+  const int m = t & 31, j = t >> 5;
+  if (m < M) {
+    double a = 0.0;
+    for (int r = j; r < R; r += 32) a += part[r * M + m];
+    slice[j][m] = a;
+  }
+  __syncthreads();
+  if (t < 32) {
     double fp = 0.0;
-    if (lane < M) {
+    if (t < M) {
       double tot = 0.0;
-      for (int w = 0; w < 8; ++w) tot += part[w][lane];
-      fp = ((double)counts[lane] / (double)N) * (tot / (double)N);
+      for (int jj = 0; jj < 32; ++jj) tot += slice[jj][t];
+      fp = ((double)counts[t] / (double)N) * (tot / (double)N);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) fp += __shfl_xor_sync(0xffffffffu, fp, off);
-    if (lane == 0) *loss = (double)alpha * (double)M * fp;
+    if (t == 0) *loss = (double)alpha * (double)M * fp;
   }
 }
 
 }  // namespace mean_detail
 
-int route_blocks(int64_t N, int M);
+int route_partial_rows(int64_t N);
 
 }  // namespace moga
 
@@ -100,7 +123,7 @@ extern "C" moga_status moga_balance_loss(const int32_t* counts, const void* rout
   if (!counts || !route_ws || !loss) return fail(MOGA_ERR_INVALID_ARG, "moga_balance_loss: null pointer");
   if (N <= 0 || N > INT32_MAX) return fail(MOGA_ERR_INVALID_ARG, "moga_balance_loss: N=%lld out of range", (long long)N);
   if (M < 1 || M > 32) return fail(MOGA_ERR_INVALID_ARG, "moga_balance_loss: M=%d not in [1, 32]", M);
-  mean_detail::balance_loss_kernel<<<1, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      counts, static_cast<const float*>(route_ws), route_blocks(N, M), (int)N, M, alpha, loss);
+  mean_detail::balance_loss_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(
+      counts, static_cast<const float*>(route_ws), route_partial_rows(N), (int)N, M, alpha, loss);
   return check_launch("moga_balance_loss");
 }

@@ -1,5 +1,5 @@
 // Router kernel: r = x . W_r (+ bias), p = softmax(r), g = argmax p, gate = p_g,
-// plus per-block partial sums of p(i|x) for the group-balancing loss.
+// plus per-chunk (32-token) partial sums of p(i|x) for the group-balancing loss.
 //
 // MoGA note (papernotes.org ICLR 2026), key design 1: a linear projection
 // with softmax gating gives p(i|x); the token goes to the most probable
@@ -20,6 +20,7 @@
 //   * logits accumulate in fp32 registers, the eight partial sums of a token
 //     are combined with three shuffles.
 #include "common.cuh"
+#include "route_tc.cu"
 
 namespace moga {
 namespace route_detail {
@@ -58,12 +59,12 @@ struct Vec<float> {
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
 __device__ __forceinline__ float to_f32(float v) { return v; }
 
-// TT tokens per thread (strided by kTokens inside the block): every W_r value
+// TT tokens per thread (strided by 4 inside the warp's 16): every W_r value
 // read from shared memory feeds TT tokens, which keeps the shared-memory
 // traffic per byte of x below the HBM rate.
 template <int MP>
 struct Tokens {
-  static constexpr int value = MP <= 8 ? 4 : 2;
+  static constexpr int value = 4;   // 128 tokens per block: 8 partial rows per 128 tokens
 };
 
 template <typename T, int MP>
@@ -73,18 +74,20 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
              int32_t* __restrict__ group_id, float* __restrict__ gate_prob,
              float* __restrict__ psum_partial) {
   constexpr int TT = Tokens<MP>::value;
-  constexpr int U = 2;   // 16-byte chunks of each token loaded ahead
+  constexpr int U = MP <= 8 ? 2 : 1;   // 16-byte chunks of each token loaded ahead
   extern __shared__ float4 smem_f4[];
   float* ws = reinterpret_cast<float*>(smem_f4);   // [MP][KC]
-  __shared__ float red[kThreads / 32][MP];
 
   const int tid = threadIdx.x;
   const int sub = tid & (kSub - 1);
-  const int tok0 = blockIdx.x * kTokens * TT + tid / kSub;
+  const int lane = tid & 31, warp = tid >> 5;
+  // warp w owns the 16 tokens [16w, 16w + 16) of the block's 128; thread
+  // (lane / 8) of a warp's token slots takes tokens lane/8 + 4t
+  const int tok0 = blockIdx.x * kTokens * TT + 16 * warp + (lane >> 3);
   const T* xrow[TT];
 #pragma unroll
   for (int t = 0; t < TT; ++t) {
-    const int tok = tok0 + t * kTokens;
+    const int tok = tok0 + 4 * t;
     xrow[t] = x + (size_t)(tok < N ? tok : 0) * d;
   }
 
@@ -150,7 +153,7 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
   for (int m = 0; m < MP; ++m) psum[m] = 0.f;
 #pragma unroll
   for (int t = 0; t < TT; ++t) {
-    const int tok = tok0 + t * kTokens;
+    const int tok = tok0 + 4 * t;
     // combine the eight partial logits of the token
 #pragma unroll
     for (int m = 0; m < MP; ++m) {
@@ -182,8 +185,9 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
     }
   }
 
-  // fixed-order block reduction of p(i|x): warp butterfly, then warps in order
-  const int lane = tid & 31, warp = tid >> 5;
+  // fixed-order sums of p(i|x) per 32-token chunk (warps 2j and 2j+1 hold
+  // chunk j of the block): one partial row per chunk, the layout the loss reads
+  __shared__ float red[kThreads / 32][MP];
 #pragma unroll
   for (int m = 0; m < MP; ++m) {
     float v = psum[m];
@@ -192,12 +196,9 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
     if (lane == 0) red[warp][m] = v;
   }
   __syncthreads();
-  if (tid < M) {
-    float sacc = 0.f;
-#pragma unroll
-    for (int w = 0; w < kThreads / 32; ++w) sacc += red[w][tid];
-    psum_partial[(size_t)blockIdx.x * M + tid] = sacc;
-  }
+  const int chunk = blockIdx.x * 4 + (warp >> 1);
+  if ((warp & 1) == 0 && lane < M && chunk * 32 < N)
+    psum_partial[(size_t)chunk * M + lane] = red[warp][lane] + red[warp + 1][lane];
 }
 
 template <typename T, int MP>
@@ -232,18 +233,19 @@ moga_status dispatch(const void* x, const void* w_r, const float* bias, int N, i
 
 }  // namespace route_detail
 
-// Blocks of the route launch for (N, M): the Σp partials have one row per block.
-int route_blocks(int64_t N, int M) {
-  const int mp = (M + 3) / 4 * 4;
-  const int tt = mp <= 8 ? 4 : 2;
-  return ceil_div((int)N, route_detail::kTokens * tt);
+// Rows of Σp partials in the route workspace: one per 32-token chunk (both
+// the tensor-core path and the fp32 path write exactly these rows).
+int route_partial_rows(int64_t N) { return ceil_div((int)N, 32); }
+
+static size_t route_partial_bytes(int64_t N, int M) {
+  return ((size_t)route_partial_rows(N) * (size_t)M * sizeof(float) + 255) / 256 * 256;
 }
 
 }  // namespace moga
 
-extern "C" size_t moga_route_ws_bytes(int64_t N, int32_t M) {
-  if (N <= 0 || N > INT32_MAX || M < 1 || M > 32) return 0;
-  return (size_t)moga::route_blocks(N, M) * (size_t)M * sizeof(float);
+extern "C" size_t moga_route_ws_bytes(int64_t N, int32_t d, int32_t M) {
+  if (N <= 0 || N > INT32_MAX || M < 1 || M > 32 || d <= 0 || d % 8 != 0) return 0;
+  return moga::route_partial_bytes(N, M) + moga::route_tc::wt_bytes(d);
 }
 
 extern "C" moga_status moga_route(const void* x, const void* w_r, moga_dtype dt, const float* bias,
@@ -256,10 +258,15 @@ extern "C" moga_status moga_route(const void* x, const void* w_r, moga_dtype dt,
   if (dt != MOGA_F32 && dt != MOGA_BF16) return fail(MOGA_ERR_INVALID_ARG, "moga_route: bad dtype %d", (int)dt);
   if (d <= 0 || d % 8 != 0) return fail(MOGA_ERR_INVALID_ARG, "moga_route: d=%d must be a positive multiple of 8", d);
   if ((reinterpret_cast<uintptr_t>(x) & 15) != 0) return fail(MOGA_ERR_INVALID_ARG, "moga_route: x not 16-byte aligned");
-  if (ws_bytes < moga_route_ws_bytes(N, M)) return fail(MOGA_ERR_WORKSPACE, "moga_route: workspace %zu < %zu bytes", ws_bytes, moga_route_ws_bytes(N, M));
+  const size_t need = moga_route_ws_bytes(N, d, M);
+  if (ws_bytes < need) return fail(MOGA_ERR_WORKSPACE, "moga_route: workspace %zu < %zu bytes", ws_bytes, need);
+  if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(MOGA_ERR_INVALID_ARG, "moga_route: workspace not 256-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   float* partial = static_cast<float*>(ws);
-  if (dt == MOGA_BF16)
-    return route_detail::dispatch<__nv_bfloat16>(x, w_r, bias, (int)N, d, M, group_id, gate_prob, partial, s);
+  if (dt == MOGA_BF16) {
+    // tensor-core path; W_r^T scratch after the partial rows
+    void* wt = static_cast<uint8_t*>(ws) + route_partial_bytes(N, M);
+    return route_tc::launch(x, w_r, bias, (int)N, d, M, group_id, gate_prob, partial, wt, 4000000000LL, s);
+  }
   return route_detail::dispatch<float>(x, w_r, bias, (int)N, d, M, group_id, gate_prob, partial, s);
 }

@@ -38,9 +38,13 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_workspace_sizes(lib):
-    assert lib.moga_route_ws_bytes(0, 5) == 0
-    assert lib.moga_route_ws_bytes(1000, 33) == 0
-    assert lib.moga_route_ws_bytes(32760, 5) == 256 * 5 * 4
+    assert lib.moga_route_ws_bytes(0, 1536, 5) == 0
+    assert lib.moga_route_ws_bytes(1000, 1536, 33) == 0
+    assert lib.moga_route_ws_bytes(1000, 12, 4) == 0
+    # one partial row per 32 tokens (256-byte aligned) + W_r^T padded to 32 groups x 64-multiple of d
+    assert lib.moga_route_ws_bytes(32760, 1536, 5) == 1024 * 5 * 4 + 32 * 1536 * 2
+    assert lib.moga_route_ws_bytes(100, 72, 3) == 256 + 32 * 128 * 2
+    assert lib.moga_route_ws_bytes(33, 8, 32) == 256 + 32 * 64 * 2
     assert lib.moga_permute_ws_bytes(32760, 5) == 2 * 16 * 5 * 4
     assert lib.moga_permute_ws_bytes(-1, 5) == 0
 

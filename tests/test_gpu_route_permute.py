@@ -28,6 +28,16 @@ CASES = {
                           win_h=1, win_w=1),
     "edge_f32_ragged": W.Workload("edge_f32", T=3, h=7, w=9, d=24, H=1, hd=64, M=5, shots=(3,), tg_max=0,
                                   win_h=7, win_w=9, x_dtype="f32"),
+    # fp32 path over many 128-token blocks, ragged last block, d not a multiple of 64, M > 16
+    "f32_blocks_M20": W.Workload("f32_blocks", T=4, h=17, w=19, d=136, H=1, hd=64, M=20, shots=(4,), tg_max=0,
+                                 win_h=17, win_w=19, x_dtype="f32"),
+    # bf16 tensor-core path: 151 chunks of 32 tokens (more chunks than SMs, so
+    # some CTAs take two), ragged last chunk, ragged last k slice, 32-column MMA
+    "bf16_chunks_M17": W.Workload("bf16_chunks", T=5, h=31, w=31, d=200, H=1, hd=64, M=17, shots=(5,),
+                                  tg_max=0, win_h=31, win_w=31),
+    # bf16, M = 16 (largest 16-column MMA), fewer chunks than SMs
+    "bf16_M16": W.Workload("bf16_M16", T=2, h=9, w=11, d=1024, H=1, hd=64, M=16, shots=(2,), tg_max=0,
+                           win_h=9, win_w=11),
 }
 
 
