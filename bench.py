@@ -37,6 +37,15 @@ WORKLOAD = W.WAN13B_5S
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM bytes (read + write) of one moga_group_attn call on the 5 s Wan-1.3B
+# workload, from an ncu --set full capture of this bench command:
+# gather3_kernel<0> 302.1 + 264.7 MB, attn_kernel<128> (MoGA launch)
+# 304.4 + 164.1 MB.  Set to None whenever either kernel changes, until it is
+# captured again.
+CALL_TRAFFIC_BYTES = 1.0352e9
+CALL_TRAFFIC_SOURCE = "ncu dram__bytes_read.sum + dram__bytes_write.sum, gather3_kernel<0> + attn_kernel<128> MoGA launch"
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -369,7 +378,8 @@ def run_ours(args):
                      "kernel": "moga_group_attn call = gather3_kernel (segment-order copy) + attn_kernel<128>",
                      "achieved": achieved,
                      "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
-                     "peak_kind": "%s burst dense bf16" % pk_kind, "traffic": None,
+                     "peak_kind": "%s burst dense bf16" % pk_kind, "traffic": CALL_TRAFFIC_BYTES,
+                     "traffic_source": CALL_TRAFFIC_SOURCE,
                      "flops_per_launch": fl_moga, "launch_ms": moga_avg_s * 1e3},
         "layer_tflops": (fl_moga + fl_stga) / (job_ms / args.steps / 1000.0) / 1e12,
         "breakdown_ms": {name: statistics.median(v) for name, v in call_ms.items()},

@@ -49,7 +49,7 @@ constexpr int BN = 128;        // key/value rows per tile
 constexpr int kThreads = 384;  // 12 warps: two softmax warpgroups + producer, MMA and two idle warps
 // Register split (setmaxnreg): the kernel launches at 168 registers per
 // thread (384 x 168 = 64512); the producer/MMA warpgroup gives back down to
-// 56 and the two softmax warpgroups take 224: 128 x 56 + 256 x 224 = 64512.
+// 120 and the two softmax warpgroups take 192: 128 x 120 + 256 x 192 = 64512.
 constexpr int kLaunchRegs = 168;
 constexpr int kSoftmaxRegs = 192;
 constexpr int kControlRegs = 120;
@@ -89,58 +89,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^x on the FMA pipe, used for a quarter of the softmax exponentials so the
-// SFU (ex2) and the FMA pipe share the load.  Method: x = n + f with n the
-// nearest integer (taken from the low mantissa bits of x + 1.5*2^23) and
-// f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose coefficients were fitted
-// here by iteratively reweighted least squares on the relative error
-// (max relative error 7.5e-5 on [-1/2, 1/2], below the bf16 rounding of P);
-// 2^n is added into the exponent field.  x is clamped to >= -126 so the
-// exponent never wraps (2^-126 is negligible next to the row sum >= 1).
-#ifndef MOGA_POLY_EXP2
-#define MOGA_POLY_EXP2 0
-#endif
-constexpr float kExp2C0 = 0.99992806f;
-constexpr float kExp2C1 = 0.69326097f;
-constexpr float kExp2C2 = 0.24261114f;
-constexpr float kExp2C3 = 0.05517166f;
-__device__ __forceinline__ float poly_exp2(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// Two exponentials with one SFU op: the pair of exponents is rounded to
-// f16x2 and ex2.approx.f16x2 returns both powers of two.  The inputs are
-// <= 8 (the reference max trails the true max by at most 2^8), so f16
-// keeps them to within 2^-7 absolute (within 2^-10 relative to the result
-// for the exponents near 0 that carry the softmax mass); the results are
-// rounded to bf16 for the P.V product anyway.
-#ifndef MOGA_SOFTMAX_X2
-#define MOGA_SOFTMAX_X2 1
-#endif
-#ifndef MOGA_P_TRUNC
-#define MOGA_P_TRUNC 0
-#endif
-#ifndef MOGA_EXP2_F16X2
-#define MOGA_EXP2_F16X2 0
-#endif
-__device__ __forceinline__ void exp2_pair(float xa, float xb, float& ea, float& eb) {
-#if MOGA_EXP2_F16X2
-  uint32_t h, e;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(xb), "f"(xa));   // xa -> low half
-  asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(h));
-  __half2 r = *reinterpret_cast<__half2*>(&e);
-  ea = __low2float(r);
-  eb = __high2float(r);
-#else
-  ea = fast_exp2(xa);
-  eb = fast_exp2(xb);
-#endif
 }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
@@ -542,14 +490,10 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
         ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + qt), sc & 1, abort_flag, timeout));
         if (!ok) break;
         tc_fence_after();
-#if MOGA_SOFTMAX_X2
         // scores as pairs, so the scale-and-shift and the row sum run as
         // packed f32x2 operations (half the instructions)
         float2 s2[BN / 2];
         float* s = reinterpret_cast<float*>(s2);
-#else
-        float s[BN];
-#endif
 #pragma unroll
         for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(s_addr + cc * 32, s + cc * 32);
         tmem_wait_ld();
@@ -575,7 +519,6 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
         const float m_old = m_run;
         if (j == 0 || need) m_run = m_new;
         const float neg_m = -m_run;
-#if MOGA_SOFTMAX_X2
         const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(neg_m, neg_m);
         float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
@@ -593,41 +536,6 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
         }
         const float2 acc01 = __fadd2_rn(acc2[0], acc2[1]), acc23 = __fadd2_rn(acc2[2], acc2[3]);
         const float row_sum = (acc01.x + acc01.y) + (acc23.x + acc23.y);
-#else
-        float sp[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
-#pragma unroll
-        for (int cc = 0; cc < BN / 16; ++cc) {
-          uint32_t pk[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float xa = fmaf(s[cc * 16 + 2 * e], sl, neg_m);
-            const float xb = fmaf(s[cc * 16 + 2 * e + 1], sl, neg_m);
-            float a, b;
-            if (MOGA_POLY_EXP2 && (e & 1)) {
-              a = fast_exp2(xa);
-              b = poly_exp2(xb);
-            } else {
-              exp2_pair(xa, xb, a, b);
-            }
-#if MOGA_P_TRUNC
-            // P rounded toward zero to bf16 by keeping the high halves (an
-            // ALU byte permute instead of a conversion), and the row sum taken
-            // over the same truncated values, so numerator and denominator of
-            // the softmax use identical weights
-            const uint32_t ua = __float_as_uint(a) & 0xFFFF0000u;
-            const uint32_t ub = __float_as_uint(b) & 0xFFFF0000u;
-            sp[e & 3] += __uint_as_float(ua) + __uint_as_float(ub);
-            pk[e] = __byte_perm(ua, ub, 0x7632);
-#else
-            sp[e & 3] += a + b;
-            pk[e] = pack_bf16x2(a, b);
-#endif
-          }
-          // P overwrites S columns [8cc, 8cc+8), whose scores were read above
-          tmem_st8(s_addr + cc * 8, pk);
-        }
-        const float row_sum = (sp[0] + sp[1]) + (sp[2] + sp[3]);
-#endif
         if (__any_sync(0xffffffffu, need)) {
           // P.V of tile j-1 finished before S of tile j (issue order), so O
           // may be rescaled here, before P_j is released to the MMA warp
