@@ -278,7 +278,10 @@ def run_ours(args):
     gs, keep = moga.geom_struct(geom)
     scale = 1.0 / math.sqrt(hd)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    CALLS = ("route", "permute", "moga_group_attn", "stga_attn", "visual_attn_mean", "moga_balance_loss")
+    if args.unfused_mean:
+        CALLS = ("route", "permute", "moga_group_attn", "stga_attn", "visual_attn_mean", "moga_balance_loss")
+    else:
+        CALLS = ("route", "permute", "moga_group_attn", "stga_attn_mean", "moga_balance_loss")
     evl = [torch.cuda.Event(enable_timing=True) for _ in range(len(CALLS) + 1)]
 
     def step(xd, qd, kd, vd, timed=False):
@@ -296,17 +299,24 @@ def run_ours(args):
         c(L.moga_group_attn(P(qd), P(kd), P(vd), N, H, hd, P(perm), P(cu), M, P(gate), scale, P(o_acc), P(aws),
                             aws.numel(), sp), "moga")
         mark(3)
-        c(L.stga_attn(P(qd), P(kd), P(vd), H, hd, moga.ctypes.byref(gs), scale, P(o_acc), P(aws), aws.numel(),
-                      sp), "stga")
-        mark(4)
-        c(L.visual_attn_mean(P(o_acc), o_acc.numel(), P(out), sp), "mean")
-        mark(5)
+        if args.unfused_mean:
+            c(L.stga_attn(P(qd), P(kd), P(vd), H, hd, moga.ctypes.byref(gs), scale, P(o_acc), P(aws), aws.numel(),
+                          sp), "stga")
+            mark(4)
+            c(L.visual_attn_mean(P(o_acc), o_acc.numel(), P(out), sp), "mean")
+        else:
+            # the three-way mean taken inside the frame pass of STGA
+            c(L.stga_attn_mean(P(qd), P(kd), P(vd), H, hd, moga.ctypes.byref(gs), scale, P(o_acc), P(out), P(aws),
+                               aws.numel(), sp), "stga_mean")
+        mark(len(CALLS) - 1)
         c(L.moga_balance_loss(P(counts), P(rws), N, M, wl.alpha, P(loss), sp), "loss")
-        mark(6)
+        mark(len(CALLS))
 
     # route 2 (W_r^T copy + tensor-core router), permute 3, MoGA gather + attention 2,
-    # STGA gather + window + frame 3, mean 1 (+tail), loss 1
-    launches_per_step = 2 + 3 + 2 + 3 + 1 + 1 + (1 if (N * H * hd) % 8 else 0)
+    # STGA gather + window + frame 3, loss 1 (+ mean 1 and its tail when not fused)
+    launches_per_step = 2 + 3 + 2 + 3 + 1
+    if args.unfused_mean:
+        launches_per_step += 1 + (1 if (N * H * hd) % 8 else 0)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -383,7 +393,8 @@ def run_ours(args):
                      "flops_per_launch": fl_moga, "launch_ms": moga_avg_s * 1e3},
         "layer_tflops": (fl_moga + fl_stga) / (job_ms / args.steps / 1000.0) / 1e12,
         "breakdown_ms": {name: statistics.median(v) for name, v in call_ms.items()},
-        "stga_tflops": fl_stga / (statistics.median(call_ms["stga_attn"]) / 1000.0) / 1e12,
+        "stga_tflops": fl_stga / (statistics.median(call_ms[CALLS[3]]) / 1000.0) / 1e12,
+        "mean_fused_into_stga": not args.unfused_mean,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
@@ -409,6 +420,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--unfused-mean", action="store_true",
+                    help="run stga_attn + visual_attn_mean instead of stga_attn_mean")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

@@ -164,6 +164,19 @@ moga_status stga_attn(const void* q, const void* k, const void* v, int32_t H, in
                       const moga_stga_geom* geom, float softmax_scale,
                       float* o_acc, void* ws, size_t ws_bytes, void* stream);
 
+/* STGA with the three-way mean fused into its last pass (note, flowchart
+ * "多组输出取均值"): the window branch adds into o_acc as in stga_attn, then
+ * the per-frame pass writes
+ *   out[t] = bf16_rn((o_acc[t] + o_frame[t]) / 3)
+ * instead of adding o_frame into o_acc, so no separate mean pass runs.  With
+ * o_acc = o_moga on entry this is the layer output, equal to
+ * stga_attn + visual_attn_mean up to the order of the fp32 additions.
+ * out: [N][H][hd] bf16, 16-byte aligned.  On return o_acc holds
+ * o_moga + o_win (the frame term is not added to it). */
+moga_status stga_attn_mean(const void* q, const void* k, const void* v, int32_t H, int32_t hd,
+                           const moga_stga_geom* geom, float softmax_scale,
+                           float* o_acc, void* out, void* ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------- mean --
  * Three-way mean (note, flowchart "多组输出取均值" and key design 4):
  *   out[i] = bf16_rn(o_acc[i] / 3) for i < n_elems, where o_acc already

@@ -9,6 +9,8 @@ kernels do every step of the layer:
     o = moga_group_attn(q, k, v, perm, cu, gate, M) # MoGA groups (o = ...)
     stga_attn(q, k, v, geom, o_acc=o)               # windows + frames (o += ...)
     out = visual_attn_mean(o)                       # bf16 (o / 3)
+    # or, mean fused into the frame pass:
+    # out = stga_attn_mean(q, k, v, geom, o_acc=o)
     loss = moga_balance_loss(counts, ws, N, M, a)   # L_gb (fp64 scalar)
 
 `visual_attention_forward` chains the six calls.
@@ -22,7 +24,7 @@ import torch
 
 from ._lib import MOGA_BF16, MOGA_F32, MogaError, StgaGeom, check, lib  # noqa: F401
 
-__all__ = ["moga_route", "moga_permute", "moga_group_attn", "stga_attn", "visual_attn_mean",
+__all__ = ["moga_route", "moga_permute", "moga_group_attn", "stga_attn", "stga_attn_mean", "visual_attn_mean",
            "moga_balance_loss", "visual_attention_forward", "attn_workspace", "device_status", "MogaError", "geom_struct"]
 
 
@@ -144,6 +146,23 @@ def stga_attn(q, k, v, geom: dict, softmax_scale: float | None = None, o_acc: to
     return o_acc
 
 
+def stga_attn_mean(q, k, v, geom: dict, o_acc: torch.Tensor, softmax_scale: float | None = None,
+                   out: torch.Tensor | None = None, ws: torch.Tensor | None = None):
+    """out = bf16((o_acc + window-group attention + per-frame attention) / 3), mean fused into the frame pass."""
+    N, H, hd = _check_qkv(q, k, v)
+    _need(o_acc, torch.float32, "o_acc", 3)
+    if out is None:
+        out = torch.empty((N, H, hd), dtype=torch.bfloat16, device=q.device)
+    _need(out, torch.bfloat16, "out", 3)
+    scale = 1.0 / math.sqrt(hd) if softmax_scale is None else softmax_scale
+    s, keep = geom_struct(geom)
+    ws = attn_workspace(q) if ws is None else ws
+    check(lib().stga_attn_mean(_ptr(q), _ptr(k), _ptr(v), H, hd, ctypes.byref(s), scale, _ptr(o_acc), _ptr(out),
+                               _ptr(ws), ws.numel(), _stream()), "stga_attn_mean")
+    del keep
+    return out
+
+
 def visual_attn_mean(o_acc: torch.Tensor, out: torch.Tensor | None = None):
     """out = bf16(o_acc / 3)."""
     _need(o_acc, torch.float32, "o_acc")
@@ -170,13 +189,19 @@ def device_status():
 
 
 def visual_attention_forward(x, w_r, bias, q, k, v, M: int, geom: dict, alpha: float,
-                             softmax_scale: float | None = None):
-    """The whole layer: returns dict(out bf16 [N,H,hd], loss fp64 [1], g, gate, perm, cu_seqlens, counts)."""
+                             softmax_scale: float | None = None, fused_mean: bool = True):
+    """The whole layer: returns dict(out bf16 [N,H,hd], loss fp64 [1], g, gate, perm, cu_seqlens, counts).
+
+    fused_mean=True takes the mean inside the STGA frame pass (stga_attn_mean);
+    False runs stga_attn then visual_attn_mean."""
     g, gate, ws = moga_route(x, w_r, bias)
     perm, cu, counts, mx = moga_permute(g, M)
     ws_attn = attn_workspace(q)
     o = moga_group_attn(q, k, v, perm, cu, gate, M, softmax_scale, ws=ws_attn)
-    stga_attn(q, k, v, geom, softmax_scale, o_acc=o, ws=ws_attn)
-    out = visual_attn_mean(o)
+    if fused_mean:
+        out = stga_attn_mean(q, k, v, geom, o, softmax_scale, ws=ws_attn)
+    else:
+        stga_attn(q, k, v, geom, softmax_scale, o_acc=o, ws=ws_attn)
+        out = visual_attn_mean(o)
     loss = moga_balance_loss(counts, ws, x.shape[0], M, alpha)
     return dict(out=out, loss=loss, g=g, gate=gate, perm=perm, cu_seqlens=cu, counts=counts, max_seqlen=mx)

@@ -74,6 +74,9 @@ struct Params {
   const float* gate;
   // output accumulator [N][H][hd]
   float* o_acc;
+  // frame launch of stga_attn_mean: out = bf16((o_acc + o_frame) / 3)
+  // instead of adding into o_acc
+  __nv_bfloat16* out;
   // STGA geometry
   int T, h, w, win_h, win_w, n_wx, n_win, whw, hw;
   int n_tg;
@@ -485,6 +488,16 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
       if (!t.valid) break;
       if (qt == 1 && !(t.q_begin + BM < t.q_end)) continue;   // no second query tile here
       const int n_kv = ceil_div(t.kv_end - t.kv_begin, BN);
+      if (p.out != nullptr) {
+        // the fused mean reads this row of the accumulator in the epilogue:
+        // start bringing it into L2 now, a whole work tile ahead
+        const int q_pre = t.q_begin + qt * BM + row;
+        if (q_pre < t.q_end) {
+          const char* a = reinterpret_cast<const char*>(p.o_acc + ((size_t)token_of(p, q_pre) * p.H + t.head) * HD);
+#pragma unroll
+          for (int e = 0; e < HD * 4; e += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(a + e));
+        }
+      }
       float m_run = -INFINITY, l_run = 0.f;
       for (int j = 0; j < n_kv; ++j, ++sc) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + qt), sc & 1, abort_flag, timeout));
@@ -578,6 +591,20 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
 #pragma unroll
           for (int e = 0; e < HD / 4; ++e)
             d4[e] = make_float4(o[4 * e] * scale, o[4 * e + 1] * scale, o[4 * e + 2] * scale, o[4 * e + 3] * scale);
+        } else if (p.out != nullptr) {
+          // last branch of the layer: the three-way mean, fused (the frames
+          // partition the tokens, so this thread owns the row)
+          // product and sum rounded separately (no FMA contraction), as in
+          // the reduction-then-mean path, so both give identical bits
+          uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)tok * p.H + t.head) * HD);
+          auto avg = [&](float acc, float v) { return __fadd_rn(acc, __fmul_rn(v, scale)) / 3.0f; };
+#pragma unroll
+          for (int e = 0; e < HD / 8; ++e) {
+            const float4 a = d4[2 * e], b = d4[2 * e + 1];
+            const float* oe = o + 8 * e;
+            dst[e] = make_uint4(pack_bf16x2(avg(a.x, oe[0]), avg(a.y, oe[1])), pack_bf16x2(avg(a.z, oe[2]), avg(a.w, oe[3])),
+                                pack_bf16x2(avg(b.x, oe[4]), avg(b.y, oe[5])), pack_bf16x2(avg(b.z, oe[6]), avg(b.w, oe[7])));
+          }
         } else {
           // the static branches add into the accumulator with fire-and-forget
           // vector reductions (each element is updated by exactly one thread
@@ -779,9 +806,9 @@ extern "C" moga_status moga_group_attn(const void* q, const void* k, const void*
   return dispatch_attn(prm, tiles, hd, w, w + bytes, w + 2 * bytes, s);
 }
 
-extern "C" moga_status stga_attn(const void* q, const void* k, const void* v, int32_t H, int32_t hd,
-                                 const moga_stga_geom* geom, float softmax_scale, float* o_acc, void* ws,
-                                 size_t ws_bytes, void* stream) {
+static moga_status stga_impl(const void* q, const void* k, const void* v, int32_t H, int32_t hd,
+                             const moga_stga_geom* geom, float softmax_scale, float* o_acc, void* out, void* ws,
+                             size_t ws_bytes, void* stream) {
   if (!geom || !geom->shot_len) return fail(MOGA_ERR_INVALID_ARG, "stga_attn: null geometry");
   const moga_stga_geom& g = *geom;
   if (g.T <= 0 || g.h <= 0 || g.w <= 0 || g.win_h <= 0 || g.win_w <= 0 || g.n_shots <= 0 || g.tg_max < 0 ||
@@ -797,6 +824,8 @@ extern "C" moga_status stga_attn(const void* q, const void* k, const void* v, in
   const int64_t N = (int64_t)g.T * g.h * g.w;
   moga_status st = check_common(q, k, v, N, H, hd, o_acc, ws, ws_bytes, true, "stga_attn");
   if (st != MOGA_OK) return st;
+  if (out && (reinterpret_cast<uintptr_t>(out) & 15))
+    return fail(MOGA_ERR_INVALID_ARG, "stga_attn_mean: out must be 16-byte aligned");
   if (!(softmax_scale > 0.f)) return fail(MOGA_ERR_INVALID_ARG, "stga_attn: softmax_scale must be > 0");
   std::vector<TGroup> tgs;
   build_temporal_groups(g, tgs);
@@ -836,5 +865,19 @@ extern "C" moga_status stga_attn(const void* q, const void* k, const void* v, in
   st = dispatch_attn(prm, prm.tg_tiles[prm.n_tg], hd, w, w + bytes, w + 2 * bytes, s);
   if (st != MOGA_OK) return st;
   prm.mode = MODE_FRAME;
+  prm.out = static_cast<__nv_bfloat16*>(out);
   return dispatch_attn(prm, g.T * H * ceil_div(prm.hw, 2 * BM), hd, q, k, v, s);
+}
+
+extern "C" moga_status stga_attn(const void* q, const void* k, const void* v, int32_t H, int32_t hd,
+                                 const moga_stga_geom* geom, float softmax_scale, float* o_acc, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  return stga_impl(q, k, v, H, hd, geom, softmax_scale, o_acc, nullptr, ws, ws_bytes, stream);
+}
+
+extern "C" moga_status stga_attn_mean(const void* q, const void* k, const void* v, int32_t H, int32_t hd,
+                                      const moga_stga_geom* geom, float softmax_scale, float* o_acc, void* out,
+                                      void* ws, size_t ws_bytes, void* stream) {
+  if (!out) return fail(MOGA_ERR_INVALID_ARG, "stga_attn_mean: null out");
+  return stga_impl(q, k, v, H, hd, geom, softmax_scale, o_acc, out, ws, ws_bytes, stream);
 }

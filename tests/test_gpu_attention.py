@@ -47,8 +47,12 @@ def _run_gpu(case, q_scale=1.0):
     o_static_cpu = o_static.cpu().numpy()
     res = moga.visual_attention_forward(t["x"], t["w_r"], t["bias"], t["q"], t["k"], t["v"], case.wl.M,
                                         case.geom, case.wl.alpha)
+    res_unfused = moga.visual_attention_forward(t["x"], t["w_r"], t["bias"], t["q"], t["k"], t["v"], case.wl.M,
+                                                case.geom, case.wl.alpha, fused_mean=False)
     moga.device_status()
     out = res["out"].float().cpu().numpy()
+    # bf16 bit patterns of the fused and the two-call output
+    _run_gpu.last_bits = (res["out"].view(torch.int16).cpu().numpy(), res_unfused["out"].view(torch.int16).cpu().numpy())
     return o_moga_cpu, o_static_cpu, out
 
 
@@ -64,23 +68,31 @@ def small(request, cuda_device):
         frame=oatt.grouped(q, k, v, ostga.frame_groups(case.geom), scale),
     )
     ref["out"] = olayer.mean3(ref["moga"], ref["win"], ref["frame"])
-    return case, ref, _run_gpu(case)
+    res = _run_gpu(case)
+    return case, ref, res, _run_gpu.last_bits
 
 
 def test_moga_attention_small(small):
-    case, ref, (o_moga, _, _) = small
+    case, ref, (o_moga, _, _), _ = small
     assert_close(o_moga, ref["moga"], "moga " + case.wl.name)
 
 
 def test_stga_attention_small(small):
-    case, ref, (_, o_static, _) = small
+    case, ref, (_, o_static, _), _ = small
     assert_close(o_static, ref["win"] + ref["frame"], "stga " + case.wl.name)
 
 
 def test_layer_output_small(small):
-    case, ref, (_, _, out) = small
+    case, ref, (_, _, out), _ = small
     # the output is bf16: add its half-ulp rounding to the budget through the same tolerance
     assert_close(out, ref["out"], "layer " + case.wl.name)
+
+
+def test_fused_mean_equals_two_calls(small):
+    """stga_attn_mean adds the frame term and divides by 3 in the same fp32 order as
+    stga_attn + visual_attn_mean, so the bf16 outputs agree bit for bit."""
+    case, _, _, (fused, unfused) = small
+    assert np.array_equal(fused, unfused), case.wl.name
 
 
 def test_peaky_queries(cuda_device):

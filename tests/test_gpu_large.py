@@ -87,12 +87,16 @@ def test_full_size_sampled(wl, cuda_device):
     tt = torch.from_numpy(toks).to(dev)
     hh = list(HEADS)
     o_m = o[tt][:, hh].cpu().numpy()
+    o_fused = o.clone()
     moga.stga_attn(q, k, v, W.stga_shape(wl), o_acc=o, ws=ws)
     o_ms = o[tt][:, hh].cpu().numpy()
     out = moga.visual_attn_mean(o)
     out_s = out[tt][:, hh].float().cpu().numpy()
+    # the mean fused into the frame pass gives the same bf16 output bit for bit
+    out_f = moga.stga_attn_mean(q, k, v, W.stga_shape(wl), o_acc=o_fused, ws=ws)
     moga.device_status()
-    del o, out, ws, q, k, v, x
+    assert torch.equal(out_f.view(torch.int16), out.view(torch.int16)), wl.name
+    del o, o_fused, out, out_f, ws, q, k, v, x
 
     scale = 1.0 / np.sqrt(wl.hd)
     wgroups = ostga.window_groups(W.stga_shape(wl))
