@@ -39,10 +39,10 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes (read + write) of one moga_group_attn call on the 5 s Wan-1.3B
 # workload, from an ncu --set full capture of this bench command:
-# gather3_kernel<0> 302.1 + 264.7 MB, attn_kernel<128> (MoGA launch)
-# 304.4 + 164.1 MB.  Set to None whenever either kernel changes, until it is
+# gather3_kernel<0> 302.1 + 263.1 MB, attn_kernel<128> (MoGA launch)
+# 305.1 + 162.2 MB.  Set to None whenever either kernel changes, until it is
 # captured again.
-CALL_TRAFFIC_BYTES = 1.0352e9
+CALL_TRAFFIC_BYTES = 1.0325e9
 CALL_TRAFFIC_SOURCE = "ncu dram__bytes_read.sum + dram__bytes_write.sum, gather3_kernel<0> + attn_kernel<128> MoGA launch"
 
 
@@ -53,6 +53,21 @@ def peaks():
         return p, "measured"
     except OSError:
         return PEAKS_FALLBACK, "fallback"
+
+
+def route_permute_hbm(wl, call_ms, pk):
+    """Algorithmic bytes of the router (x once, g and gate out, one Σp row per 32 tokens)
+    and of the permute (g in, perm out; counts and cu are negligible) over their
+    CUDA-event call times, as a fraction of the measured HBM copy bandwidth."""
+    xb = 2 if wl.x_dtype == "bf16" else 4
+    route_b = wl.N * wl.d * xb + 8 * wl.N + 4 * wl.M * (-(-wl.N // 32))
+    perm_b = 8 * wl.N + 8 * (wl.M + 1)
+    out = {}
+    for name, b in (("route", route_b), ("permute", perm_b)):
+        ms = statistics.median(call_ms[name])
+        gbs = b / (ms * 1e-3) / 1e9
+        out[name] = {"bytes": b, "ms": ms, "gbs": gbs, "frac": gbs / pk["hbm_gbs"]}
+    return out
 
 
 def moga_flops(counts, H, hd):
@@ -278,7 +293,7 @@ def run_ours(args):
     gs, keep = moga.geom_struct(geom)
     scale = 1.0 / math.sqrt(hd)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    if args.unfused_mean:
+    if not args.fused_mean:
         CALLS = ("route", "permute", "moga_group_attn", "stga_attn", "visual_attn_mean", "moga_balance_loss")
     else:
         CALLS = ("route", "permute", "moga_group_attn", "stga_attn_mean", "moga_balance_loss")
@@ -299,7 +314,7 @@ def run_ours(args):
         c(L.moga_group_attn(P(qd), P(kd), P(vd), N, H, hd, P(perm), P(cu), M, P(gate), scale, P(o_acc), P(aws),
                             aws.numel(), sp), "moga")
         mark(3)
-        if args.unfused_mean:
+        if not args.fused_mean:
             c(L.stga_attn(P(qd), P(kd), P(vd), H, hd, moga.ctypes.byref(gs), scale, P(o_acc), P(aws), aws.numel(),
                           sp), "stga")
             mark(4)
@@ -315,7 +330,7 @@ def run_ours(args):
     # route 2 (W_r^T copy + tensor-core router), permute 3, MoGA gather + attention 2,
     # STGA gather + window + frame 3, loss 1 (+ mean 1 and its tail when not fused)
     launches_per_step = 2 + 3 + 2 + 3 + 1
-    if args.unfused_mean:
+    if not args.fused_mean:
         launches_per_step += 1 + (1 if (N * H * hd) % 8 else 0)
 
     for _ in range(args.warmup):
@@ -394,7 +409,8 @@ def run_ours(args):
         "layer_tflops": (fl_moga + fl_stga) / (job_ms / args.steps / 1000.0) / 1e12,
         "breakdown_ms": {name: statistics.median(v) for name, v in call_ms.items()},
         "stga_tflops": fl_stga / (statistics.median(call_ms[CALLS[3]]) / 1000.0) / 1e12,
-        "mean_fused_into_stga": not args.unfused_mean,
+        "mean_fused_into_stga": bool(args.fused_mean),
+        "route_permute_hbm": route_permute_hbm(wl, call_ms, pk),
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
@@ -420,8 +436,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--unfused-mean", action="store_true",
-                    help="run stga_attn + visual_attn_mean instead of stga_attn_mean")
+    ap.add_argument("--fused-mean", action="store_true",
+                    help="run stga_attn_mean (mean inside the STGA frame pass) instead of stga_attn + visual_attn_mean")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
