@@ -195,6 +195,93 @@ moga_status visual_attn_mean(const float* o_acc, int64_t n_elems, void* out, voi
 moga_status moga_balance_loss(const int32_t* counts, const void* route_ws, int64_t N, int32_t M,
                               float alpha, double* loss, void* stream);
 
+/* =============================================================== training
+ * Forward calls that keep what the backward needs, and the backward of the
+ * layer (MoGA note, key designs 1 and 3: the layer is trained end to end; the
+ * gate p(g(x)|x) on the MoGA output is the router's path to a gradient, and
+ * L_gb is added to the objective).  The backward differentiates
+ *   J = sum(dout * out) + dloss * L_gb
+ * with g(x) = argmax and the counts treated as constants (zero gradient).
+ * Q, K, V are inputs of the layer: their projection from x is outside it, so
+ * x receives gradient through the router only.  Conventions as above
+ * (device pointers, caller-owned buffers, asynchronous on `stream`). */
+
+/* moga_route plus probs [N][M] fp32 out: p(i|x_t), the softmax the backward
+ * differentiates. */
+moga_status moga_route_train(const void* x, const void* w_r, moga_dtype dt, const float* bias,
+                             int64_t N, int32_t d, int32_t M, int32_t* group_id, float* gate_prob,
+                             float* probs, void* ws, size_t ws_bytes, void* stream);
+
+/* moga_group_attn plus lse [N][H] fp32 out: the log-sum-exp of each row's
+ * scaled scores in log2 units (lse = log2 sum_j 2^(q.k_j * scale * log2 e)),
+ * so that P = 2^(q.k * scale * log2 e - lse).  o_moga is written as in
+ * moga_group_attn (gate * attention). */
+moga_status moga_group_attn_train(const void* q, const void* k, const void* v,
+                                  int64_t N, int32_t H, int32_t hd,
+                                  const int32_t* perm, const int32_t* cu_seqlens, int32_t M,
+                                  const float* gate_prob, float softmax_scale,
+                                  float* o_moga, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* STGA with the two static branches kept apart: o_win and o_frame
+ * [N][H][hd] fp32 are WRITTEN (each token is a query of exactly one window
+ * group and one frame), lse_win / lse_frame [N][H] fp32 as above. */
+moga_status stga_attn_train(const void* q, const void* k, const void* v, int32_t H, int32_t hd,
+                            const moga_stga_geom* geom, float softmax_scale,
+                            float* o_win, float* lse_win, float* o_frame, float* lse_frame,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* out[i] = bf16_rn(((o_moga[i] + o_win[i]) + o_frame[i]) / 3); n_elems % 4 == 0,
+ * 16-byte aligned pointers. */
+moga_status visual_attn_mean3(const float* o_moga, const float* o_win, const float* o_frame,
+                              int64_t n_elems, void* out, void* stream);
+
+/* Attention backward workspace: Q, K, V and dout copied into segment order
+ * plus per-row statistics; 256-byte aligned, at least this many bytes.
+ * Returns 0 for arguments the calls would reject. */
+size_t moga_attn_bwd_ws_bytes(int64_t N, int32_t H, int32_t hd);
+
+/* Backward of the MoGA branch.  Per group and head, with S = Q K^T * scale,
+ * P = softmax(S), O = P V and the branch's upstream gradient
+ * dO = gate * dout / 3:  dV = P^T dO, dS = P * (dO V^T - rowsum(dO * O)),
+ * dQ = dS K * scale, dK = dS^T Q * scale;  dgate[t] = sum_{h,d} dout/3 * O.
+ * o_moga, lse: from moga_group_attn_train;  dout [N][H][hd] bf16;
+ * dq, dk, dv [N][H][hd] fp32: ADDED TO (all three branches accumulate);
+ * dgate [N] fp32: written. */
+moga_status moga_group_attn_bwd(const void* q, const void* k, const void* v,
+                                int64_t N, int32_t H, int32_t hd,
+                                const int32_t* perm, const int32_t* cu_seqlens, int32_t M,
+                                const float* gate_prob, float softmax_scale,
+                                const float* o_moga, const float* lse, const void* dout,
+                                float* dq, float* dk, float* dv, float* dgate,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* Backward of the two static branches (window groups with their
+ * adjacent-shot frames, and frames), dO = dout / 3 for each; keys shared by
+ * two window groups receive both contributions.  o_win, lse_win, o_frame,
+ * lse_frame: from stga_attn_train;  dq, dk, dv: ADDED TO. */
+moga_status stga_attn_bwd(const void* q, const void* k, const void* v, int32_t H, int32_t hd,
+                          const moga_stga_geom* geom, float softmax_scale,
+                          const float* o_win, const float* lse_win,
+                          const float* o_frame, const float* lse_frame, const void* dout,
+                          float* dq, float* dk, float* dv, void* ws, size_t ws_bytes, void* stream);
+
+/* Router backward workspace (per-block partial sums of dW_r); 256-byte
+ * aligned.  Returns 0 for arguments moga_route_bwd would reject. */
+size_t moga_route_bwd_ws_bytes(int64_t N, int32_t d, int32_t M);
+
+/* Router backward through the gate and the balancing loss:
+ *   u[t][m] = dgate[t] * [m == g_t] + dloss * alpha * M * (counts[m] / N) / N,
+ *   dr[t] = p_t * (u[t] - <u[t], p_t>),
+ *   dx = dr W_r^T ([N][d] fp32, written), dW_r = x^T dr ([d][M] fp32, written),
+ *   dbias = sum_t dr[t] ([M] fp32, written; NULL to skip).
+ * x, w_r: as for moga_route (dtype dt);  group_id, probs: from
+ * moga_route_train;  dgate: from moga_group_attn_bwd;  counts: from
+ * moga_permute;  dloss: the objective's weight on L_gb. */
+moga_status moga_route_bwd(const void* x, const void* w_r, moga_dtype dt, int64_t N, int32_t d, int32_t M,
+                           const int32_t* group_id, const float* probs, const float* dgate,
+                           const int32_t* counts, float alpha, float dloss,
+                           float* dx, float* dw_r, float* dbias, void* ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------- diagnostics */
 /* Text of the last host-side error of the calling thread ("" if none). */
 const char* moga_last_error(void);

@@ -25,7 +25,8 @@ import torch
 from ._lib import MOGA_BF16, MOGA_F32, MogaError, StgaGeom, check, lib  # noqa: F401
 
 __all__ = ["moga_route", "moga_permute", "moga_group_attn", "stga_attn", "stga_attn_mean", "visual_attn_mean",
-           "moga_balance_loss", "visual_attention_forward", "attn_workspace", "device_status", "MogaError", "geom_struct"]
+           "moga_balance_loss", "visual_attention_forward", "attn_workspace", "device_status", "MogaError", "geom_struct",
+           "visual_attention_forward_train", "visual_attention_backward"]
 
 
 def _ptr(t):
@@ -205,3 +206,82 @@ def visual_attention_forward(x, w_r, bias, q, k, v, M: int, geom: dict, alpha: f
         out = visual_attn_mean(o)
     loss = moga_balance_loss(counts, ws, x.shape[0], M, alpha)
     return dict(out=out, loss=loss, g=g, gate=gate, perm=perm, cu_seqlens=cu, counts=counts, max_seqlen=mx)
+
+
+# ---------------------------------------------------------------- training
+#
+# The training forward keeps the router probabilities, the three branch
+# outputs and each branch's per-row log-sum-exp; the backward differentiates
+# J = sum(dout * out) + dloss * L_gb (argmax and counts are constants).
+
+def visual_attention_forward_train(x, w_r, bias, q, k, v, M: int, geom: dict, alpha: float,
+                                   softmax_scale: float | None = None):
+    """Forward that saves what the backward needs.  Returns dict(out, loss, saved)."""
+    L = lib()
+    N, d = x.shape
+    _, H, hd = _check_qkv(q, k, v)
+    dev = x.device
+    scale = 1.0 / math.sqrt(hd) if softmax_scale is None else softmax_scale
+    rws = torch.empty(max(L.moga_route_ws_bytes(N, d, M), 16), dtype=torch.uint8, device=dev)
+    g = torch.empty(N, dtype=torch.int32, device=dev)
+    gate = torch.empty(N, dtype=torch.float32, device=dev)
+    probs = torch.empty((N, M), dtype=torch.float32, device=dev)
+    dt = MOGA_BF16 if x.dtype == torch.bfloat16 else MOGA_F32
+    check(L.moga_route_train(_ptr(x), _ptr(w_r), dt, _ptr(bias), N, d, M, _ptr(g), _ptr(gate), _ptr(probs),
+                             _ptr(rws), rws.numel(), _stream()), "moga_route_train")
+    perm, cu, counts, mx = moga_permute(g, M)
+    ws = attn_workspace(q)
+    f32 = dict(dtype=torch.float32, device=dev)
+    o_moga, o_win, o_frame = (torch.empty((N, H, hd), **f32) for _ in range(3))
+    lse_moga, lse_win, lse_frame = (torch.empty((N, H), **f32) for _ in range(3))
+    check(L.moga_group_attn_train(_ptr(q), _ptr(k), _ptr(v), N, H, hd, _ptr(perm), _ptr(cu), M, _ptr(gate), scale,
+                                  _ptr(o_moga), _ptr(lse_moga), _ptr(ws), ws.numel(), _stream()),
+          "moga_group_attn_train")
+    s, keep = geom_struct(geom)
+    check(L.stga_attn_train(_ptr(q), _ptr(k), _ptr(v), H, hd, ctypes.byref(s), scale, _ptr(o_win), _ptr(lse_win),
+                            _ptr(o_frame), _ptr(lse_frame), _ptr(ws), ws.numel(), _stream()), "stga_attn_train")
+    del keep
+    out = torch.empty((N, H, hd), dtype=torch.bfloat16, device=dev)
+    check(L.visual_attn_mean3(_ptr(o_moga), _ptr(o_win), _ptr(o_frame), out.numel(), _ptr(out), _stream()),
+          "visual_attn_mean3")
+    loss = moga_balance_loss(counts, rws, N, M, alpha)
+    saved = dict(g=g, gate=gate, probs=probs, perm=perm, cu_seqlens=cu, counts=counts, o_moga=o_moga,
+                 lse_moga=lse_moga, o_win=o_win, lse_win=lse_win, o_frame=o_frame, lse_frame=lse_frame,
+                 scale=scale)
+    return dict(out=out, loss=loss, saved=saved)
+
+
+def visual_attention_backward(saved: dict, x, w_r, q, k, v, M: int, geom: dict, alpha: float, dout, dloss: float,
+                              with_bias: bool = False):
+    """Gradients of sum(dout * out) + dloss * L_gb.  dout [N, H, hd] bf16.
+
+    Returns dict(dq, dk, dv [N, H, hd] fp32, dx [N, d] fp32, dw_r [d, M] fp32,
+    dbias [M] fp32 or None, dgate [N] fp32)."""
+    L = lib()
+    N, d = x.shape
+    _, H, hd = _check_qkv(q, k, v)
+    _need(dout, torch.bfloat16, "dout", 3)
+    dev = q.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.zeros((N, H, hd), **f32) for _ in range(3))
+    dgate = torch.empty(N, **f32)
+    ws = torch.empty(L.moga_attn_bwd_ws_bytes(N, H, hd), dtype=torch.uint8, device=dev)
+    sc = saved["scale"]
+    check(L.moga_group_attn_bwd(_ptr(q), _ptr(k), _ptr(v), N, H, hd, _ptr(saved["perm"]), _ptr(saved["cu_seqlens"]),
+                                M, _ptr(saved["gate"]), sc, _ptr(saved["o_moga"]), _ptr(saved["lse_moga"]),
+                                _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgate), _ptr(ws), ws.numel(),
+                                _stream()), "moga_group_attn_bwd")
+    s, keep = geom_struct(geom)
+    check(L.stga_attn_bwd(_ptr(q), _ptr(k), _ptr(v), H, hd, ctypes.byref(s), sc, _ptr(saved["o_win"]),
+                          _ptr(saved["lse_win"]), _ptr(saved["o_frame"]), _ptr(saved["lse_frame"]), _ptr(dout),
+                          _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream()), "stga_attn_bwd")
+    del keep
+    dx = torch.empty((N, d), **f32)
+    dw_r = torch.empty((d, M), **f32)
+    dbias = torch.empty(M, **f32) if with_bias else None
+    rws = torch.empty(L.moga_route_bwd_ws_bytes(N, d, M), dtype=torch.uint8, device=dev)
+    dt = MOGA_BF16 if x.dtype == torch.bfloat16 else MOGA_F32
+    check(L.moga_route_bwd(_ptr(x), _ptr(w_r), dt, N, d, M, _ptr(saved["g"]), _ptr(saved["probs"]), _ptr(dgate),
+                           _ptr(saved["counts"]), alpha, dloss, _ptr(dx), _ptr(dw_r), _ptr(dbias), _ptr(rws),
+                           rws.numel(), _stream()), "moga_route_bwd")
+    return dict(dq=dq, dk=dk, dv=dv, dx=dx, dw_r=dw_r, dbias=dbias, dgate=dgate)

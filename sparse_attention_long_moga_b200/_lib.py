@@ -32,6 +32,18 @@ SIGNATURES = {
     "stga_attn_mean": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _P, _F32, _P, _P, _P, _SZ, _P]),
     "visual_attn_mean": (ctypes.c_int, [_P, _I64, _P, _P]),
     "moga_balance_loss": (ctypes.c_int, [_P, _P, _I64, _I32, _F32, _P, _P]),
+    "moga_route_train": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _I64, _I32, _I32, _P, _P, _P, _P, _SZ, _P]),
+    "moga_group_attn_train": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I32, _P, _P, _I32, _P, _F32, _P, _P, _P, _SZ,
+                                             _P]),
+    "stga_attn_train": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _P, _F32, _P, _P, _P, _P, _P, _SZ, _P]),
+    "visual_attn_mean3": (ctypes.c_int, [_P, _P, _P, _I64, _P, _P]),
+    "moga_attn_bwd_ws_bytes": (_SZ, [_I64, _I32, _I32]),
+    "moga_group_attn_bwd": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I32, _P, _P, _I32, _P, _F32, _P, _P, _P, _P, _P,
+                                           _P, _P, _P, _SZ, _P]),
+    "stga_attn_bwd": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _P, _F32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moga_route_bwd_ws_bytes": (_SZ, [_I64, _I32, _I32]),
+    "moga_route_bwd": (ctypes.c_int, [_P, _P, ctypes.c_int, _I64, _I32, _I32, _P, _P, _P, _P, _F32, _F32, _P, _P, _P,
+                                      _P, _SZ, _P]),
     "moga_last_error": (ctypes.c_char_p, []),
     "moga_device_status": (ctypes.c_int, [_P]),
     "moga_version": (ctypes.c_char_p, []),

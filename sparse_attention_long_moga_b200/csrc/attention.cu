@@ -77,6 +77,12 @@ struct Params {
   // frame launch of stga_attn_mean: out = bf16((o_acc + o_frame) / 3)
   // instead of adding into o_acc
   __nv_bfloat16* out;
+  // training forward: per-row log2-domain log-sum-exp of the scaled scores,
+  // lse[t][h] = m + log2(l) so that P = 2^(s * scale * log2(e) - lse) ([N][H]
+  // fp32, optional), and the static branches write their own output instead
+  // of adding into a shared accumulator
+  float* lse;
+  int write_static;
   // STGA geometry
   int T, h, w, win_h, win_w, n_wx, n_win, whw, hw;
   int n_tg;
@@ -139,7 +145,9 @@ struct GroupTable {
   int prefix[33];   // CTA-tile prefix over the ordered groups
 };
 
-__device__ void build_group_table(const Params& p, GroupTable& gt) {
+// unit_rows: query rows per work unit (two 128-row tiles in the forward, one
+// in the backward)
+__device__ void build_group_table(const Params& p, GroupTable& gt, int unit_rows = 2 * BM) {
   int size[32], order[32];
   for (int i = 0; i < p.M; ++i) {
     size[i] = __ldg(p.cu + i + 1) - __ldg(p.cu + i);
@@ -160,7 +168,7 @@ __device__ void build_group_table(const Params& p, GroupTable& gt) {
     const int g = order[k];
     gt.start[k] = __ldg(p.cu + g);
     gt.size[k] = size[g];
-    gt.prefix[k + 1] = gt.prefix[k] + ceil_div(size[g], 2 * BM) * p.H;
+    gt.prefix[k + 1] = gt.prefix[k] + ceil_div(size[g], unit_rows) * p.H;
   }
 }
 
@@ -587,7 +595,8 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
         float scale = 1.0f / l_run;
         if (p.mode == MODE_MOGA) scale *= __ldg(p.gate + tok);
         float4* d4 = reinterpret_cast<float4*>(p.o_acc + ((size_t)tok * p.H + t.head) * HD);
-        if (p.mode == MODE_MOGA) {
+        if (p.lse != nullptr) p.lse[(size_t)tok * p.H + t.head] = m_run + log2f(l_run);
+        if (p.mode == MODE_MOGA || p.write_static) {
 #pragma unroll
           for (int e = 0; e < HD / 4; ++e)
             d4[e] = make_float4(o[4 * e] * scale, o[4 * e + 1] * scale, o[4 * e + 2] * scale, o[4 * e + 3] * scale);
@@ -776,10 +785,10 @@ extern "C" size_t moga_attn_ws_bytes(int64_t N, int32_t H, int32_t hd) {
   return attn_ws_bytes(N, H, hd);
 }
 
-extern "C" moga_status moga_group_attn(const void* q, const void* k, const void* v, int64_t N, int32_t H, int32_t hd,
-                                       const int32_t* perm, const int32_t* cu_seqlens, int32_t M,
-                                       const float* gate_prob, float softmax_scale, float* o_acc, void* ws,
-                                       size_t ws_bytes, void* stream) {
+static moga_status moga_impl(const void* q, const void* k, const void* v, int64_t N, int32_t H, int32_t hd,
+                             const int32_t* perm, const int32_t* cu_seqlens, int32_t M, const float* gate_prob,
+                             float softmax_scale, float* o_acc, float* lse, void* ws, size_t ws_bytes,
+                             void* stream) {
   moga_status st = check_common(q, k, v, N, H, hd, o_acc, ws, ws_bytes, true, "moga_group_attn");
   if (st != MOGA_OK) return st;
   if (!perm || !cu_seqlens || !gate_prob) return fail(MOGA_ERR_INVALID_ARG, "moga_group_attn: null pointer");
@@ -796,6 +805,7 @@ extern "C" moga_status moga_group_attn(const void* q, const void* k, const void*
   prm.M = M;
   prm.gate = gate_prob;
   prm.o_acc = o_acc;
+  prm.lse = lse;
   fill_debug(prm);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((st = launch_gather(prm, hd, q, k, v, ws, s)) != MOGA_OK) return st;
@@ -806,38 +816,50 @@ extern "C" moga_status moga_group_attn(const void* q, const void* k, const void*
   return dispatch_attn(prm, tiles, hd, w, w + bytes, w + 2 * bytes, s);
 }
 
-static moga_status stga_impl(const void* q, const void* k, const void* v, int32_t H, int32_t hd,
-                             const moga_stga_geom* geom, float softmax_scale, float* o_acc, void* out, void* ws,
-                             size_t ws_bytes, void* stream) {
-  if (!geom || !geom->shot_len) return fail(MOGA_ERR_INVALID_ARG, "stga_attn: null geometry");
+extern "C" moga_status moga_group_attn(const void* q, const void* k, const void* v, int64_t N, int32_t H, int32_t hd,
+                                       const int32_t* perm, const int32_t* cu_seqlens, int32_t M,
+                                       const float* gate_prob, float softmax_scale, float* o_acc, void* ws,
+                                       size_t ws_bytes, void* stream) {
+  return moga_impl(q, k, v, N, H, hd, perm, cu_seqlens, M, gate_prob, softmax_scale, o_acc, nullptr, ws, ws_bytes,
+                   stream);
+}
+
+extern "C" moga_status moga_group_attn_train(const void* q, const void* k, const void* v, int64_t N, int32_t H,
+                                             int32_t hd, const int32_t* perm, const int32_t* cu_seqlens, int32_t M,
+                                             const float* gate_prob, float softmax_scale, float* o_moga, float* lse,
+                                             void* ws, size_t ws_bytes, void* stream) {
+  if (!lse) return fail(MOGA_ERR_INVALID_ARG, "moga_group_attn_train: null lse");
+  return moga_impl(q, k, v, N, H, hd, perm, cu_seqlens, M, gate_prob, softmax_scale, o_moga, lse, ws, ws_bytes,
+                   stream);
+}
+
+// Validates the STGA geometry and fills the static-branch fields of prm
+// (temporal groups, window tiling, tile prefix); N = T*h*w.
+static moga_status stga_params(const moga_stga_geom* geom, int32_t H, float softmax_scale, Params& prm,
+                               int64_t& N, const char* who) {
+  if (!geom || !geom->shot_len) return fail(MOGA_ERR_INVALID_ARG, "%s: null geometry", who);
   const moga_stga_geom& g = *geom;
   if (g.T <= 0 || g.h <= 0 || g.w <= 0 || g.win_h <= 0 || g.win_w <= 0 || g.n_shots <= 0 || g.tg_max < 0 ||
       g.aug_frames < 0)
-    return fail(MOGA_ERR_INVALID_ARG, "stga_attn: bad geometry");
-  if (g.h % g.win_h || g.w % g.win_w) return fail(MOGA_ERR_INVALID_ARG, "stga_attn: windows must tile the frame");
+    return fail(MOGA_ERR_INVALID_ARG, "%s: bad geometry", who);
+  if (g.h % g.win_h || g.w % g.win_w) return fail(MOGA_ERR_INVALID_ARG, "%s: windows must tile the frame", who);
   long long tsum = 0;
   for (int s = 0; s < g.n_shots; ++s) {
-    if (g.shot_len[s] <= 0) return fail(MOGA_ERR_INVALID_ARG, "stga_attn: shot %d has length %d", s, g.shot_len[s]);
+    if (g.shot_len[s] <= 0) return fail(MOGA_ERR_INVALID_ARG, "%s: shot %d has length %d", who, s, g.shot_len[s]);
     tsum += g.shot_len[s];
   }
-  if (tsum != g.T) return fail(MOGA_ERR_INVALID_ARG, "stga_attn: shot lengths sum to %lld, T=%d", tsum, g.T);
-  const int64_t N = (int64_t)g.T * g.h * g.w;
-  moga_status st = check_common(q, k, v, N, H, hd, o_acc, ws, ws_bytes, true, "stga_attn");
-  if (st != MOGA_OK) return st;
-  if (out && (reinterpret_cast<uintptr_t>(out) & 15))
-    return fail(MOGA_ERR_INVALID_ARG, "stga_attn_mean: out must be 16-byte aligned");
-  if (!(softmax_scale > 0.f)) return fail(MOGA_ERR_INVALID_ARG, "stga_attn: softmax_scale must be > 0");
+  if (tsum != g.T) return fail(MOGA_ERR_INVALID_ARG, "%s: shot lengths sum to %lld, T=%d", who, tsum, g.T);
+  if (!(softmax_scale > 0.f)) return fail(MOGA_ERR_INVALID_ARG, "%s: softmax_scale must be > 0", who);
+  N = (int64_t)g.T * g.h * g.w;
+  if (N * (int64_t)H >= INT32_MAX) return fail(MOGA_ERR_INVALID_ARG, "%s: N*H out of range", who);
   std::vector<TGroup> tgs;
   build_temporal_groups(g, tgs);
   if ((int)tgs.size() > kMaxTG)
-    return fail(MOGA_ERR_UNSUPPORTED, "stga_attn: %zu temporal groups (max %d)", tgs.size(), kMaxTG);
-
-  Params prm;
+    return fail(MOGA_ERR_UNSUPPORTED, "%s: %zu temporal groups (max %d)", who, tgs.size(), kMaxTG);
   memset(&prm, 0, sizeof(prm));
   prm.N = (int)N;
   prm.H = H;
   prm.scale_log2 = softmax_scale * 1.4426950408889634f;
-  prm.o_acc = o_acc;
   prm.T = g.T;
   prm.h = g.h;
   prm.w = g.w;
@@ -855,29 +877,62 @@ static moga_status stga_impl(const void* q, const void* k, const void* v, int32_
     prm.tg_tiles[i + 1] = prm.tg_tiles[i] + prm.n_win * H * qp;
   }
   fill_debug(prm);
+  return MOGA_OK;
+}
+
+// o_win / o_frame: the same accumulator (added to) unless write is set, in
+// which case each branch writes its own buffer; out: fused mean (frame pass).
+static moga_status stga_impl(const void* q, const void* k, const void* v, int32_t H, int32_t hd,
+                             const moga_stga_geom* geom, float softmax_scale, float* o_win, float* o_frame,
+                             float* lse_win, float* lse_frame, bool write, void* out, void* ws, size_t ws_bytes,
+                             void* stream, const char* who) {
+  Params prm;
+  int64_t N = 0;
+  moga_status st = stga_params(geom, H, softmax_scale, prm, N, who);
+  if (st != MOGA_OK) return st;
+  if ((st = check_common(q, k, v, N, H, hd, o_win, ws, ws_bytes, true, who)) != MOGA_OK) return st;
+  if (!o_frame || (reinterpret_cast<uintptr_t>(o_frame) & 15))
+    return fail(MOGA_ERR_INVALID_ARG, "%s: frame output must be a 16-byte aligned pointer", who);
+  if (out && (reinterpret_cast<uintptr_t>(out) & 15))
+    return fail(MOGA_ERR_INVALID_ARG, "%s: out must be 16-byte aligned", who);
+  prm.write_static = write ? 1 : 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // window groups (gathered into window-major order), then frames (already
   // contiguous); both add into o_acc and stream order keeps them apart
   prm.mode = MODE_WINDOW;
+  prm.o_acc = o_win;
+  prm.lse = lse_win;
   if ((st = launch_gather(prm, hd, q, k, v, ws, s)) != MOGA_OK) return st;
   const uint8_t* w = static_cast<const uint8_t*>(ws);
   const size_t bytes = (size_t)N * H * hd * 2;
   st = dispatch_attn(prm, prm.tg_tiles[prm.n_tg], hd, w, w + bytes, w + 2 * bytes, s);
   if (st != MOGA_OK) return st;
   prm.mode = MODE_FRAME;
+  prm.o_acc = o_frame;
+  prm.lse = lse_frame;
   prm.out = static_cast<__nv_bfloat16*>(out);
-  return dispatch_attn(prm, g.T * H * ceil_div(prm.hw, 2 * BM), hd, q, k, v, s);
+  return dispatch_attn(prm, prm.T * H * ceil_div(prm.hw, 2 * BM), hd, q, k, v, s);
 }
 
 extern "C" moga_status stga_attn(const void* q, const void* k, const void* v, int32_t H, int32_t hd,
                                  const moga_stga_geom* geom, float softmax_scale, float* o_acc, void* ws,
                                  size_t ws_bytes, void* stream) {
-  return stga_impl(q, k, v, H, hd, geom, softmax_scale, o_acc, nullptr, ws, ws_bytes, stream);
+  return stga_impl(q, k, v, H, hd, geom, softmax_scale, o_acc, o_acc, nullptr, nullptr, false, nullptr, ws, ws_bytes,
+                   stream, "stga_attn");
 }
 
 extern "C" moga_status stga_attn_mean(const void* q, const void* k, const void* v, int32_t H, int32_t hd,
                                       const moga_stga_geom* geom, float softmax_scale, float* o_acc, void* out,
                                       void* ws, size_t ws_bytes, void* stream) {
   if (!out) return fail(MOGA_ERR_INVALID_ARG, "stga_attn_mean: null out");
-  return stga_impl(q, k, v, H, hd, geom, softmax_scale, o_acc, out, ws, ws_bytes, stream);
+  return stga_impl(q, k, v, H, hd, geom, softmax_scale, o_acc, o_acc, nullptr, nullptr, false, out, ws, ws_bytes,
+                   stream, "stga_attn_mean");
+}
+
+extern "C" moga_status stga_attn_train(const void* q, const void* k, const void* v, int32_t H, int32_t hd,
+                                       const moga_stga_geom* geom, float softmax_scale, float* o_win, float* lse_win,
+                                       float* o_frame, float* lse_frame, void* ws, size_t ws_bytes, void* stream) {
+  if (!lse_win || !lse_frame) return fail(MOGA_ERR_INVALID_ARG, "stga_attn_train: null lse");
+  return stga_impl(q, k, v, H, hd, geom, softmax_scale, o_win, o_frame, lse_win, lse_frame, true, nullptr, ws,
+                   ws_bytes, stream, "stga_attn_train");
 }

@@ -85,6 +85,20 @@ balance_loss_kernel(const int32_t* __restrict__ counts, const float* __restrict_
   }
 }
 
+// Training forward: the three branch outputs kept apart (for the backward);
+// out = bf16_rn((a + b) + c) / 3), 4 elements per thread per step.
+__global__ void __launch_bounds__(kThreads)
+mean3_sep_kernel(const float4* __restrict__ a, const float4* __restrict__ b, const float4* __restrict__ c,
+                 uint2* __restrict__ out, int64_t n4) {
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n4; i += stride) {
+    const float4 x = __ldcs(a + i), y = __ldcs(b + i), z = __ldcs(c + i);
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(((x.x + y.x) + z.x) / 3.0f, ((x.y + y.y) + z.y) / 3.0f);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(((x.z + y.z) + z.z) / 3.0f, ((x.w + y.w) + z.w) / 3.0f);
+    __stcs(out + i, make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi)));
+  }
+}
+
 }  // namespace mean_detail
 
 int route_partial_rows(int64_t N);
@@ -115,6 +129,27 @@ extern "C" moga_status visual_attn_mean(const float* o_acc, int64_t n_elems, voi
     return check_launch("visual_attn_mean/tail");
   }
   return MOGA_OK;
+}
+
+extern "C" moga_status visual_attn_mean3(const float* o_moga, const float* o_win, const float* o_frame,
+                                         int64_t n_elems, void* out, void* stream) {
+  using namespace moga;
+  using namespace moga::mean_detail;
+  if (!o_moga || !o_win || !o_frame || !out) return fail(MOGA_ERR_INVALID_ARG, "visual_attn_mean3: null pointer");
+  if (n_elems <= 0 || n_elems % 4) return fail(MOGA_ERR_INVALID_ARG, "visual_attn_mean3: n_elems=%lld", (long long)n_elems);
+  const uintptr_t al = reinterpret_cast<uintptr_t>(o_moga) | reinterpret_cast<uintptr_t>(o_win) |
+                       reinterpret_cast<uintptr_t>(o_frame) | reinterpret_cast<uintptr_t>(out);
+  if (al & 15) return fail(MOGA_ERR_INVALID_ARG, "visual_attn_mean3: pointers must be 16-byte aligned");
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t n4 = n_elems / 4;
+  const int blocks = (int)std::min<int64_t>(ceil_div((int)std::min<int64_t>(n4, INT32_MAX / 2), kThreads),
+                                            (int64_t)sms * 16);
+  mean3_sep_kernel<<<blocks, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const float4*>(o_moga), reinterpret_cast<const float4*>(o_win),
+      reinterpret_cast<const float4*>(o_frame), static_cast<uint2*>(out), n4);
+  return check_launch("visual_attn_mean3");
 }
 
 extern "C" moga_status moga_balance_loss(const int32_t* counts, const void* route_ws, int64_t N, int32_t M,

@@ -6,3 +6,5 @@
 #include "permute_noalloc.cu"
 #include "mean_loss.cu"
 #include "attention.cu"
+#include "attention_bwd.cu"
+#include "route_bwd.cu"

@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(kThreads)
 route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __restrict__ bias,
              int N, int d, int M, int KC,
              int32_t* __restrict__ group_id, float* __restrict__ gate_prob,
-             float* __restrict__ psum_partial) {
+             float* __restrict__ psum_partial, float* __restrict__ probs) {
   constexpr int TT = Tokens<MP>::value;
   constexpr int U = MP <= 8 ? 2 : 1;   // 16-byte chunks of each token loaded ahead
   extern __shared__ float4 smem_f4[];
@@ -182,6 +182,10 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
       for (int m = 0; m < MP; ++m) psum[m] += e[m] * inv;
       group_id[tok] = g;
       gate_prob[tok] = inv;   // exp(r_g - max) = 1
+      if (probs != nullptr)
+#pragma unroll
+        for (int m = 0; m < MP; ++m)
+          if (m < M) probs[(size_t)tok * M + m] = e[m] * inv;
     }
   }
 
@@ -203,7 +207,7 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
 
 template <typename T, int MP>
 moga_status launch(const void* x, const void* w_r, const float* bias, int N, int d, int M,
-                   int32_t* g, float* gate, float* partial, cudaStream_t s) {
+                   int32_t* g, float* gate, float* partial, float* probs, cudaStream_t s) {
   int KC = kSmemBudget / (MP * 4);
   KC = (KC / (8 * kSub)) * (8 * kSub);   // whole 8-element chunks for every thread of a token
   if (KC >= d) KC = d;
@@ -212,22 +216,22 @@ moga_status launch(const void* x, const void* w_r, const float* bias, int N, int
   if (e != cudaSuccess) return fail(MOGA_ERR_CUDA, "moga_route: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
   const int blocks = ceil_div(N, kTokens * Tokens<MP>::value);
   route_kernel<T, MP><<<blocks, kThreads, smem, s>>>(static_cast<const T*>(x), static_cast<const T*>(w_r),
-                                                     bias, N, d, M, KC, g, gate, partial);
+                                                     bias, N, d, M, KC, g, gate, partial, probs);
   return check_launch("moga_route");
 }
 
 template <typename T>
 moga_status dispatch(const void* x, const void* w_r, const float* bias, int N, int d, int M,
-                     int32_t* g, float* gate, float* partial, cudaStream_t s) {
+                     int32_t* g, float* gate, float* partial, float* probs, cudaStream_t s) {
   switch ((M + 3) / 4) {
-    case 1: return launch<T, 4>(x, w_r, bias, N, d, M, g, gate, partial, s);
-    case 2: return launch<T, 8>(x, w_r, bias, N, d, M, g, gate, partial, s);
-    case 3: return launch<T, 12>(x, w_r, bias, N, d, M, g, gate, partial, s);
-    case 4: return launch<T, 16>(x, w_r, bias, N, d, M, g, gate, partial, s);
-    case 5: return launch<T, 20>(x, w_r, bias, N, d, M, g, gate, partial, s);
-    case 6: return launch<T, 24>(x, w_r, bias, N, d, M, g, gate, partial, s);
-    case 7: return launch<T, 28>(x, w_r, bias, N, d, M, g, gate, partial, s);
-    default: return launch<T, 32>(x, w_r, bias, N, d, M, g, gate, partial, s);
+    case 1: return launch<T, 4>(x, w_r, bias, N, d, M, g, gate, partial, probs, s);
+    case 2: return launch<T, 8>(x, w_r, bias, N, d, M, g, gate, partial, probs, s);
+    case 3: return launch<T, 12>(x, w_r, bias, N, d, M, g, gate, partial, probs, s);
+    case 4: return launch<T, 16>(x, w_r, bias, N, d, M, g, gate, partial, probs, s);
+    case 5: return launch<T, 20>(x, w_r, bias, N, d, M, g, gate, partial, probs, s);
+    case 6: return launch<T, 24>(x, w_r, bias, N, d, M, g, gate, partial, probs, s);
+    case 7: return launch<T, 28>(x, w_r, bias, N, d, M, g, gate, partial, probs, s);
+    default: return launch<T, 32>(x, w_r, bias, N, d, M, g, gate, partial, probs, s);
   }
 }
 
@@ -248,9 +252,11 @@ extern "C" size_t moga_route_ws_bytes(int64_t N, int32_t d, int32_t M) {
   return moga::route_partial_bytes(N, M) + moga::route_tc::wt_bytes(d);
 }
 
-extern "C" moga_status moga_route(const void* x, const void* w_r, moga_dtype dt, const float* bias,
-                                  int64_t N, int32_t d, int32_t M, int32_t* group_id, float* gate_prob,
-                                  void* ws, size_t ws_bytes, void* stream) {
+namespace moga {
+
+static moga_status route_impl(const void* x, const void* w_r, moga_dtype dt, const float* bias, int64_t N, int32_t d,
+                              int32_t M, int32_t* group_id, float* gate_prob, float* probs, void* ws,
+                              size_t ws_bytes, void* stream) {
   using namespace moga;
   if (!x || !w_r || !group_id || !gate_prob || !ws) return fail(MOGA_ERR_INVALID_ARG, "moga_route: null pointer");
   if (N <= 0 || N > INT32_MAX) return fail(MOGA_ERR_INVALID_ARG, "moga_route: N=%lld out of range", (long long)N);
@@ -266,7 +272,22 @@ extern "C" moga_status moga_route(const void* x, const void* w_r, moga_dtype dt,
   if (dt == MOGA_BF16) {
     // tensor-core path; W_r^T scratch after the partial rows
     void* wt = static_cast<uint8_t*>(ws) + route_partial_bytes(N, M);
-    return route_tc::launch(x, w_r, bias, (int)N, d, M, group_id, gate_prob, partial, wt, 4000000000LL, s);
+    return route_tc::launch(x, w_r, bias, (int)N, d, M, group_id, gate_prob, partial, probs, wt, 4000000000LL, s);
   }
-  return route_detail::dispatch<float>(x, w_r, bias, (int)N, d, M, group_id, gate_prob, partial, s);
+  return route_detail::dispatch<float>(x, w_r, bias, (int)N, d, M, group_id, gate_prob, partial, probs, s);
+}
+
+}  // namespace moga
+
+extern "C" moga_status moga_route(const void* x, const void* w_r, moga_dtype dt, const float* bias,
+                                  int64_t N, int32_t d, int32_t M, int32_t* group_id, float* gate_prob,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  return moga::route_impl(x, w_r, dt, bias, N, d, M, group_id, gate_prob, nullptr, ws, ws_bytes, stream);
+}
+
+extern "C" moga_status moga_route_train(const void* x, const void* w_r, moga_dtype dt, const float* bias,
+                                        int64_t N, int32_t d, int32_t M, int32_t* group_id, float* gate_prob,
+                                        float* probs, void* ws, size_t ws_bytes, void* stream) {
+  if (!probs) return moga::fail(MOGA_ERR_INVALID_ARG, "moga_route_train: null probs");
+  return moga::route_impl(x, w_r, dt, bias, N, d, M, group_id, gate_prob, probs, ws, ws_bytes, stream);
 }

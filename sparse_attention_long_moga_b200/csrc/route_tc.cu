@@ -82,6 +82,7 @@ struct Params {
   int32_t* group_id;
   float* gate_prob;
   float* partial;      // [n_chunks][M]: sum of p(i|x) over the chunk's tokens
+  float* probs;        // [N][M] p(i|x) (training forward) or null
   long long timeout;
 };
 
@@ -255,6 +256,10 @@ route_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
         for (int m = 0; m < NP; ++m) pr[m] *= inv;
         p.group_id[tok] = g;
         p.gate_prob[tok] = inv;   // exp(r_g - max) = 1
+        if (p.probs != nullptr)
+#pragma unroll
+          for (int m = 0; m < NP; ++m)
+            if (m < p.M) p.probs[(size_t)tok * p.M + m] = pr[m];
       } else {
 #pragma unroll
         for (int m = 0; m < NP; ++m) pr[m] = 0.f;
@@ -335,7 +340,7 @@ static moga_status launch_np(const Params& prm, const void* wt, int dpad, const 
 
 // x [N][d] bf16, w_r [d][M] bf16; partial [ceil(N/32)][M]; wt scratch of wt_bytes(d).
 moga_status launch(const void* x, const void* w_r, const float* bias, int N, int d, int M, int32_t* g, float* gate,
-                   float* partial, void* wt, long long timeout, cudaStream_t s) {
+                   float* partial, float* probs, void* wt, long long timeout, cudaStream_t s) {
   const int dpad = dpad_of(d);
   prep_wt_kernel<<<ceil_div(NPMAX * dpad, 256), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w_r), d, M, dpad,
                                                             static_cast<__nv_bfloat16*>(wt));
@@ -351,6 +356,7 @@ moga_status launch(const void* x, const void* w_r, const float* bias, int N, int
   prm.group_id = g;
   prm.gate_prob = gate;
   prm.partial = partial;
+  prm.probs = probs;
   prm.timeout = timeout;
   return M <= 16 ? launch_np<16>(prm, wt, dpad, x, s) : launch_np<32>(prm, wt, dpad, x, s);
 }

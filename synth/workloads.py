@@ -32,7 +32,7 @@ import numpy as np
 from . import rng
 
 # counter streams
-S_X, S_WR, S_Q, S_K, S_V, S_WQ, S_WK, S_WV, S_MU, S_EPS, S_REGION = range(1, 12)
+S_X, S_WR, S_Q, S_K, S_V, S_WQ, S_WK, S_WV, S_MU, S_EPS, S_REGION, S_DOUT = range(1, 13)
 
 
 @dataclass(frozen=True)
@@ -237,6 +237,13 @@ def qkv_stored(wl: Workload, which: str, redraw: dict | None = None, chunk: int 
         out[a:b] = qkv_rows_bits(wl, which, np.arange(a, b), redraw)
     _parallel_chunks(wl.N, chunk, fill)
     return out
+
+
+def dout_bits(wl: Workload) -> np.ndarray:
+    """bf16 bits of an upstream gradient of the layer output, i.i.d. N(0, 1): [N, H, hd]."""
+    width = wl.H * wl.hd
+    idx = np.arange(wl.N, dtype=np.uint64)[:, None] * np.uint64(width) + np.arange(width, dtype=np.uint64)[None, :]
+    return to_bf16_bits(rng.normal(wl.seed, S_DOUT, idx)).reshape(wl.N, wl.H, wl.hd)
 
 
 def stga_shape(wl: Workload) -> dict:

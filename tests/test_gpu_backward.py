@@ -1,0 +1,75 @@
+"""GPU parity of the layer backward against the fp64 backward oracle.
+
+The objective is J = sum(dout * out) + dloss * L_gb with a seeded bf16 dout;
+both sides read the same stored inputs.  Attention gradients are products of
+bf16 operands (P and dS rounded to bf16 for the tensor core, like P in the
+forward) with fp32 accumulation, so they get the forward's rel-L2 budget
+1e-2, with the max-abs bound taken relative to the largest reference entry
+(3e-2 of it).  The router gradients (dgate, dx, dW_r, dbias) are fp32 sums of
+those and get the same budget.
+"""
+import numpy as np
+import pytest
+
+from _data import Case, rel_l2
+from oracle import backward as ob
+from synth import workloads as W
+from test_gpu_attention import SMALL
+
+pytestmark = pytest.mark.gpu
+
+REL = 1e-2
+MAXREL = 3e-2
+DLOSS = 0.5
+
+
+def _close(got, want, what):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    r = rel_l2(got, want)
+    m = float(np.max(np.abs(got - want))) if want.size else 0.0
+    scale = float(np.max(np.abs(want))) if want.size else 1.0
+    assert r <= REL and m <= MAXREL * max(scale, 1e-30), "%s: rel-L2 %.3e, max-abs %.3e (max |ref| %.3e)" % (
+        what, r, m, scale)
+
+
+@pytest.fixture(scope="module", params=sorted(SMALL))
+def grads(request, cuda_device):
+    import torch
+    import sparse_attention_long_moga_b200 as moga
+    case = Case(SMALL[request.param])
+    wl = case.wl
+    t = case.gpu()
+    dbits = W.dout_bits(wl)
+    dout = torch.from_numpy(dbits.view(np.int16)).to(cuda_device).view(torch.bfloat16)
+    fw = moga.visual_attention_forward_train(t["x"], t["w_r"], t["bias"], t["q"], t["k"], t["v"], wl.M, case.geom,
+                                             wl.alpha)
+    gb = moga.visual_attention_backward(fw["saved"], t["x"], t["w_r"], t["q"], t["k"], t["v"], wl.M, case.geom,
+                                        wl.alpha, dout, DLOSS, with_bias=t["bias"] is not None)
+    moga.device_status()
+    got = {k: (None if v is None else v.cpu().numpy()) for k, v in gb.items()}
+    got["out"] = fw["out"].float().cpu().numpy()
+    q, k, v = case.qkv64()
+    ref = ob.layer_backward(case.x64(), case.w64(), case.bias, q, k, v, wl.M, case.geom, wl.alpha,
+                            W.bf16_bits_to_f64(dbits), DLOSS)
+    return case, got, ref
+
+
+@pytest.mark.parametrize("name", ["dq", "dk", "dv"])
+def test_attention_gradients(grads, name):
+    case, got, ref = grads
+    _close(got[name], ref[name], "%s %s" % (name, case.wl.name))
+
+
+def test_gate_gradient(grads):
+    case, got, ref = grads
+    _close(got["dgate"], ref["dgate"], "dgate " + case.wl.name)
+
+
+@pytest.mark.parametrize("name", ["dx", "dw_r", "dbias"])
+def test_router_gradients(grads, name):
+    case, got, ref = grads
+    if ref[name] is None:
+        assert got[name] is None
+        return
+    _close(got[name], ref[name], "%s %s" % (name, case.wl.name))
