@@ -429,6 +429,126 @@ def run_ours(args):
     return 0
 
 
+def run_train(args):
+    """Training step on one GPU: the saving forward (route with probabilities, permute,
+    MoGA and STGA with per-branch outputs and log-sum-exp, mean, loss) followed by the
+    backward (attention branches, gate, router and loss), through the C ABI with
+    persistent buffers.  Prints one JSON line (not the forward headline line)."""
+    import torch
+
+    import sparse_attention_long_moga_b200 as moga
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    wl = WORKLOAD
+    inp = make_inputs(wl)
+    geom = W.stga_shape(wl)
+
+    def to_dev(a):
+        t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+        return t.to(dev).view(torch.bfloat16) if a.dtype == np.uint16 else t.to(dev)
+
+    x, w_r, q, k, v = (to_dev(inp[n]) for n in ("x", "w_r", "q", "k", "v"))
+    dout = torch.from_numpy(W.dout_bits(wl).view(np.int16)).to(dev).view(torch.bfloat16)
+    N, M, H, hd, d = wl.N, wl.M, wl.H, wl.hd, wl.d
+    L = moga._lib.lib()
+    sp = moga._stream()
+    P = moga._ptr
+    stream = torch.cuda.current_stream()
+    f32 = dict(dtype=torch.float32, device=dev)
+    i32 = dict(dtype=torch.int32, device=dev)
+    g, perm, counts, mx, cu = (torch.empty(n, **i32) for n in (N, N, M, 1, M + 1))
+    gate, dgate = torch.empty(N, **f32), torch.empty(N, **f32)
+    probs = torch.empty((N, M), **f32)
+    rws = torch.empty(max(L.moga_route_ws_bytes(N, d, M), 16), dtype=torch.uint8, device=dev)
+    pws = torch.empty(max(L.moga_permute_ws_bytes(N, M), 16), dtype=torch.uint8, device=dev)
+    aws = torch.empty(L.moga_attn_ws_bytes(N, H, hd), dtype=torch.uint8, device=dev)
+    bws = torch.empty(L.moga_attn_bwd_ws_bytes(N, H, hd), dtype=torch.uint8, device=dev)
+    rbws = torch.empty(L.moga_route_bwd_ws_bytes(N, d, M), dtype=torch.uint8, device=dev)
+    o_moga, o_win, o_frame, dq, dk, dv = (torch.empty((N, H, hd), **f32) for _ in range(6))
+    lse_moga, lse_win, lse_frame = (torch.empty((N, H), **f32) for _ in range(3))
+    out = torch.empty((N, H, hd), dtype=torch.bfloat16, device=dev)
+    loss = torch.empty(1, dtype=torch.float64, device=dev)
+    dx, dw_r = torch.empty((N, d), **f32), torch.empty((d, M), **f32)
+    gs, keep = moga.geom_struct(geom)
+    scale = 1.0 / math.sqrt(hd)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    CALLS = ("moga_route_train", "moga_permute", "moga_group_attn_train", "stga_attn_train", "visual_attn_mean3",
+             "moga_balance_loss", "zero_grads", "moga_group_attn_bwd", "stga_attn_bwd", "moga_route_bwd")
+
+    def step(evl=None):
+        c = moga.check
+
+        def mark(i):
+            if evl is not None:
+                evl[i].record(stream)
+        mark(0)
+        c(L.moga_route_train(P(x), P(w_r), moga.MOGA_BF16, None, N, d, M, P(g), P(gate), P(probs), P(rws),
+                             rws.numel(), sp), "route")
+        mark(1)
+        c(L.moga_permute(P(g), N, M, P(perm), P(cu), P(counts), P(mx), P(pws), pws.numel(), sp), "permute")
+        mark(2)
+        c(L.moga_group_attn_train(P(q), P(k), P(v), N, H, hd, P(perm), P(cu), M, P(gate), scale, P(o_moga),
+                                  P(lse_moga), P(aws), aws.numel(), sp), "moga")
+        mark(3)
+        c(L.stga_attn_train(P(q), P(k), P(v), H, hd, moga.ctypes.byref(gs), scale, P(o_win), P(lse_win),
+                            P(o_frame), P(lse_frame), P(aws), aws.numel(), sp), "stga")
+        mark(4)
+        c(L.visual_attn_mean3(P(o_moga), P(o_win), P(o_frame), out.numel(), P(out), sp), "mean3")
+        mark(5)
+        c(L.moga_balance_loss(P(counts), P(rws), N, M, wl.alpha, P(loss), sp), "loss")
+        mark(6)
+        for t in (dq, dk, dv):
+            t.zero_()
+        mark(7)
+        c(L.moga_group_attn_bwd(P(q), P(k), P(v), N, H, hd, P(perm), P(cu), M, P(gate), scale, P(o_moga),
+                                P(lse_moga), P(dout), P(dq), P(dk), P(dv), P(dgate), P(bws), bws.numel(), sp),
+          "moga bwd")
+        mark(8)
+        c(L.stga_attn_bwd(P(q), P(k), P(v), H, hd, moga.ctypes.byref(gs), scale, P(o_win), P(lse_win), P(o_frame),
+                          P(lse_frame), P(dout), P(dq), P(dk), P(dv), P(bws), bws.numel(), sp), "stga bwd")
+        mark(9)
+        c(L.moga_route_bwd(P(x), P(w_r), moga.MOGA_BF16, N, d, M, P(g), P(probs), P(dgate), P(counts), wl.alpha, 1.0,
+                           P(dx), P(dw_r), None, P(rbws), rbws.numel(), sp), "route bwd")
+        mark(10)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    moga.device_status()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(CALLS) + 1)] for _ in range(args.steps)]
+    sampler = ClockSampler(0)
+    torch.cuda.synchronize()
+    sampler.start()
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    moga.device_status()
+    call_ms = {name: statistics.median(e[j].elapsed_time(e[j + 1]) for e in evs) for j, name in enumerate(CALLS)}
+    step_ms = statistics.median(e[0].elapsed_time(e[-1]) for e in evs)
+    fl_fwd_moga = moga_flops(counts.cpu().numpy(), H, hd)
+    fl_fwd_stga = stga_flops(wl)
+    pk, pk_kind = peaks()
+    # attention backward FLOPs in the usual convention: 2.5 x forward (dV, dP, dQ, dK
+    # and the recomputed S; the dQ pass recomputes S and dP once more on top of that)
+    bwd_moga_tf = 2.5 * fl_fwd_moga / (call_ms["moga_group_attn_bwd"] * 1e-3) / 1e12
+    bwd_stga_tf = 2.5 * fl_fwd_stga / (call_ms["stga_attn_bwd"] * 1e-3) / 1e12
+    line = {
+        "metric": "visual-attn layer training step (fwd + bwd) tokens/s (bf16)", "value": N / (step_ms * 1e-3),
+        "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic (seeded counter-based generator; no dataset)",
+        "config": config_dict(wl), "breakdown_ms": call_ms,
+        "attn_bwd_tflops": {"moga": bwd_moga_tf, "stga": bwd_stga_tf,
+                            "moga_frac_of_peak": bwd_moga_tf / pk["bf16_tflops"],
+                            "convention": "2.5 x forward FLOPs (4*H*hd*sum n_q*n_kv)"},
+        "peak": {"bf16_tflops": pk["bf16_tflops"], "kind": pk_kind},
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -438,9 +558,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fused-mean", action="store_true",
                     help="run stga_attn_mean (mean inside the STGA frame pass) instead of stga_attn + visual_attn_mean")
+    ap.add_argument("--train", action="store_true",
+                    help="time the training step (saving forward + backward) instead of the forward")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.train:
+        return run_train(args)
     return run_ours(args)
 
 

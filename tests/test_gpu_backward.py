@@ -73,3 +73,42 @@ def test_router_gradients(grads, name):
         assert got[name] is None
         return
     _close(got[name], ref[name], "%s %s" % (name, case.wl.name))
+
+
+def test_full_size_heads(cuda_device):
+    """The 32k-token Wan-1.3B-shaped workload (the one the benchmark times): the GPU
+    backward over all 12 heads, compared on three whole heads (every token) with the
+    oracle's per-branch backward of those heads (dgate and the router gradients need
+    all heads and are covered by the small cases)."""
+    import torch
+    import sparse_attention_long_moga_b200 as moga
+    wl = W.WAN13B_5S
+    case = Case(wl, with_qkv=False)
+    redraw = case.redraw
+    qb, kb, vb = (W.qkv_stored(wl, n, redraw) for n in "qkv")
+    dbits = W.dout_bits(wl)
+
+    def up(a):
+        return torch.from_numpy(a.view(np.int16)).to(cuda_device).view(torch.bfloat16)
+    t = case.gpu()
+    q, k, v, dout = up(qb), up(kb), up(vb), up(dbits)
+    fw = moga.visual_attention_forward_train(t["x"], t["w_r"], t["bias"], q, k, v, wl.M, case.geom, wl.alpha)
+    gb = moga.visual_attention_backward(fw["saved"], t["x"], t["w_r"], q, k, v, wl.M, case.geom, wl.alpha, dout, 0.0)
+    moga.device_status()
+    heads = (0, 5, 11)
+    got = {n: gb[n][:, list(heads)].cpu().numpy() for n in ("dq", "dk", "dv")}
+    del fw, gb, q, k, v, dout
+
+    from oracle import route as oroute
+    from oracle import stga as ostga
+    g, p_g, _ = oroute.route(case.x64(), case.w64(), case.bias)
+    scale = 1.0 / np.sqrt(wl.hd)
+    for j, h in enumerate(heads):
+        qh, kh, vh = (W.bf16_bits_to_f64(a[:, h:h + 1, :]) for a in (qb, kb, vb))
+        do = W.bf16_bits_to_f64(dbits[:, h:h + 1, :]) / 3.0
+        dq, dk, dv, _ = ob.moga_bwd(qh, kh, vh, g, p_g, wl.M, scale, do)
+        for groups in (ostga.window_groups(case.geom), ostga.frame_groups(case.geom)):
+            a, b, c = ob.grouped_bwd(qh, kh, vh, do, groups, scale)
+            dq, dk, dv = dq + a, dk + b, dv + c
+        for n, ref in (("dq", dq), ("dk", dk), ("dv", dv)):
+            _close(got[n][:, j], ref[:, 0], "%s head %d %s" % (n, h, wl.name))
