@@ -20,14 +20,18 @@
 //                     per-row statistics the tiles need: the forward's
 //                     log-sum-exp, D' and c (and dgate for MoGA)
 //   bwd_dkdv_kernel   one CTA per (segment, head, 128-key tile): loops over
-//                     the segment's 128-query tiles; S^T = K Q^T and
-//                     dP^T = V dO^T on tcgen05 (keys on the TMEM lanes, so
-//                     P^T and dS^T come out as the A operand of the next two
-//                     products), then dV += (c P)^T dO and dK += dS^T Q
-//                     accumulate in TMEM; the epilogue adds them into dv, dk
-//   bwd_dq_kernel     one CTA per (segment, head, 128-query tile): loops over
-//                     the segment's key tiles; S = Q K^T, dP = dO V^T, then
-//                     dQ += dS K in TMEM; the epilogue adds into dq
+//                     the segment's queries in 64-row halves of 128-row
+//                     tiles; S^T = K Q^T and dP^T = V dO^T on tcgen05 (keys
+//                     on the TMEM lanes, so c P^T and dS^T come out as the A
+//                     operand of the next two products), then dV += (c P)^T dO
+//                     and dK += dS^T Q accumulate in TMEM; two TMEM buffers,
+//                     so the products of one half overlap the exponentials of
+//                     the other; the epilogue adds dV, dK into dv, dk
+//   bwd_dq_kernel     one CTA per (segment, head, 128-query tile): Q and dO
+//                     copied once into TMEM as bf16 pairs (the A operands of
+//                     S = Q K^T and dP = dO V^T), the segment's keys streamed
+//                     in 64-row halves, dQ += dS K in TMEM; the epilogue adds
+//                     into dq
 // Both: warps 0-3 compute (thread = TMEM lane), warp 4 TMA producer, warp 5
 // TMEM allocator and MMA issuer.  All waits are bounded.
 //
@@ -209,12 +213,14 @@ enum BwdBar : int {
   BB_RES = 0,        // resident tiles landed
   BB_FULL = 1,       // +stage: streamed tiles landed
   BB_EMPTY = 3,      // +stage: streamed tiles consumed by the MMAs
-  BB_S = 5,          // S (and dP) products in TMEM
-  BB_P = 6,          // compute wrote the bf16 operands (128 arrivals)
-  BB_DONE = 7,       // accumulators final
-  BB_END = 8,        // every MMA finished (teardown)
-  BB_COUNT = 9
+  BB_S = 5,          // +buffer: S (and dP) products of a 64-wide half tile in TMEM
+  BB_P = 7,          // +buffer: compute wrote the bf16 operands of that half (128 arrivals)
+  BB_DONE = 9,       // accumulators final
+  BB_END = 10,       // every MMA finished (teardown)
+  BB_A = 11,         // resident operands copied into TMEM (128 arrivals)
+  BB_COUNT = 12
 };
+static_assert(BB_COUNT <= BwdSmem<128>::kNumBars, "barrier area");
 
 __device__ __forceinline__ uint32_t bwd_pack(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -251,10 +257,13 @@ __device__ __forceinline__ bool bwd_setup(const BwdParams& b, uint8_t* smem, uin
       mbar_init(bar0 + 8 * (BB_FULL + s), 1);
       mbar_init(bar0 + 8 * (BB_EMPTY + s), 1);
     }
-    mbar_init(bar0 + 8 * BB_S, 1);
-    mbar_init(bar0 + 8 * BB_P, BM);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar0 + 8 * (BB_S + s), 1);
+      mbar_init(bar0 + 8 * (BB_P + s), BM);
+    }
     mbar_init(bar0 + 8 * BB_DONE, 1);
     mbar_init(bar0 + 8 * BB_END, 1);
+    mbar_init(bar0 + 8 * BB_A, BM);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -290,33 +299,76 @@ __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* map, 
   for (int hh = 0; hh < HD / 64; ++hh) tma_load_3d(dst + hh * kHalfBytes, map, hh * 64, head, r0, bar);
 }
 
-// S-type product D[128 x 128] = A[128 x HD] . B[128 x HD]^T, both K-major tiles.
+// S-type product over a 64-wide half: D[128 x 64] = A[128 x HD] . B[64 x HD]^T,
+// B the rows [64 half, 64 half + 64) of a K-major 128-row tile.
 template <int HD>
-__device__ __forceinline__ void mma_nt(uint32_t d_tmem, uint32_t a, uint32_t bt) {
-  constexpr uint32_t idesc = instr_desc(BN, false);
+__device__ __forceinline__ void mma_nt_half(uint32_t d_tmem, uint32_t a, uint32_t bt, int half) {
+  constexpr uint32_t idesc = instr_desc(BN / 2, false);
+  const uint32_t b = bt + half * (BN / 2) * 128;
 #pragma unroll
   for (int ks = 0; ks < HD / 16; ++ks) {
     const uint64_t ad = smem_desc(a + (ks >> 2) * kHalfBytes + (ks & 3) * 32, 16, 1024);
-    const uint64_t bd = smem_desc(bt + (ks >> 2) * kHalfBytes + (ks & 3) * 32, 16, 1024);
+    const uint64_t bd = smem_desc(b + (ks >> 2) * kHalfBytes + (ks & 3) * 32, 16, 1024);
     tc_mma_ss(d_tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
   }
 }
 
-// Accumulating product D[128 x HD] (+)= A[128 x 128] . B[128 x HD], A in TMEM
-// (bf16 pairs, 8 columns per 16 of K), B an MN-major tile in shared memory.
+// Accumulating product over a 64-deep half: D[128 x HD] (+)= A[128 x 64] .
+// B[64 x HD], A in TMEM (bf16 pairs, 32 columns), B the rows [64 half, ...)
+// of an MN-major 128-row tile.
 template <int HD>
-__device__ __forceinline__ void mma_tn(uint32_t d_tmem, uint32_t a_tmem, uint32_t b, bool acc) {
+__device__ __forceinline__ void mma_tn_half(uint32_t d_tmem, uint32_t a_tmem, uint32_t b, int half, bool acc) {
   constexpr uint32_t idesc = instr_desc(HD, true);
 #pragma unroll
-  for (int ks = 0; ks < BN / 16; ++ks) {
-    const uint64_t bd = smem_desc(b + ks * 16 * 128, kHalfBytes, 1024);
+  for (int ks = 0; ks < BN / 32; ++ks) {
+    const uint64_t bd = smem_desc(b + (half * (BN / 2) + ks * 16) * 128, kHalfBytes, 1024);
     tc_mma_ts(d_tmem, a_tmem + ks * 8, bd, idesc, (acc || ks > 0) ? 1u : 0u);
+  }
+}
+
+// Row `row` of a 128-row SW128 tile in shared memory (HD columns in 64-column
+// halves) into TMEM as bf16 pairs: column c holds elements 2c, 2c+1, the
+// layout of an A operand in tensor memory.  Called by the thread whose TMEM
+// lane is `row`.
+template <int HD>
+__device__ __forceinline__ void tile_row_to_tmem(const uint8_t* tile, int row, uint32_t taddr) {
+#pragma unroll
+  for (int hh = 0; hh < HD / 64; ++hh) {
+    const uint8_t* base = tile + hh * kHalfBytes + row * 128;
+    float w[32];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 v = *reinterpret_cast<const uint4*>(base + ((c ^ (row & 7)) << 4));
+      w[4 * c] = __uint_as_float(v.x);
+      w[4 * c + 1] = __uint_as_float(v.y);
+      w[4 * c + 2] = __uint_as_float(v.z);
+      w[4 * c + 3] = __uint_as_float(v.w);
+    }
+    tmem_st32(taddr + hh * 32, w);
+  }
+}
+
+// S-type product over a 64-wide half with A in TMEM: D[128 x 64] = A[128 x HD]
+// (bf16 pairs) . B[64 x HD]^T, B the rows [64 half, ...) of a K-major tile.
+// Only B is read from shared memory (2 KB per MMA instead of 6 KB).
+template <int HD>
+__device__ __forceinline__ void mma_ts_half(uint32_t d_tmem, uint32_t a_tmem, uint32_t bt, int half) {
+  constexpr uint32_t idesc = instr_desc(BN / 2, false);
+  const uint32_t b = bt + half * (BN / 2) * 128;
+#pragma unroll
+  for (int ks = 0; ks < HD / 16; ++ks) {
+    const uint64_t bd = smem_desc(b + (ks >> 2) * kHalfBytes + (ks & 3) * 32, 16, 1024);
+    tc_mma_ts(d_tmem, a_tmem + ks * 8, bd, idesc, ks > 0 ? 1u : 0u);
   }
 }
 
 // ------------------------------------------------------------------ dK, dV
 
-// TMEM: S^T [0,128), dP^T [128,256), dV [256, 256+HD), dK [256+HD, 256+2HD).
+// TMEM: two 128-column buffers for 64-query halves (S^T at +0, dP^T at +64;
+// c P^T and dS^T overwrite the first 32 columns of each), dV [256, 256 + HD),
+// dK [256 + HD, 256 + 2 HD).  K and V stay in shared memory: copying them into
+// TMEM as A operands leaves room for one buffer only at HD = 128, and the
+// exponentials then no longer overlap the products (measured slower).
 template <int HD>
 __global__ void __launch_bounds__(192, 1)
 bwd_dkdv_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUtensorMap tm_q,
@@ -346,22 +398,35 @@ bwd_dkdv_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUt
       load_tile<HD>(sbase + SM::kRes0, &tm_k, u.head, u.t_begin, bar(BB_RES));
       load_tile<HD>(sbase + SM::kRes1, &tm_v, u.head, u.t_begin, bar(BB_RES));
     }
+    // per-query statistics of a tile (lse, D', c for 128 rows, 4 per lane);
+    // rows past the segment get c = 0 and a huge log-sum-exp, so their P and
+    // dS are exactly 0.  Loaded a tile ahead, so the global-load latency
+    // overlaps the wait for the stage.
+    float pre[3][BM / 32];
+    auto fetch = [&](int i) {
+      const int r0 = u.q_begin + i * BM;
+#pragma unroll
+      for (int e = 0; e < BM / 32; ++e) {
+        const int r = r0 + lane + 32 * e;
+        const bool in = i < n_q && r < u.q_end;
+        pre[0][e] = in ? __ldg(b.lse_seg + (size_t)r * p.H + u.head) : 3.0e38f;
+        pre[1][e] = in ? __ldg(b.dd_seg + (size_t)r * p.H + u.head) : 0.f;
+        pre[2][e] = in ? __ldg(b.c_seg + r) : 0.f;
+      }
+    };
+    fetch(0);
     for (int i = 0; i < n_q && ok; ++i) {
       const int s = i & 1;
       const uint32_t ph = (i >> 1) & 1;
       ok = __shfl_sync(0xffffffffu, lane == 0 ? (int)mbar_wait(bar(BB_EMPTY + s), ph ^ 1, abort_flag, timeout) : 0, 0);
       if (!ok) break;
-      // per-query statistics of this tile; rows past the segment get c = 0 and a
-      // huge log-sum-exp, so their P and dS are exactly 0
       const int r0 = u.q_begin + i * BM;
       float* st = stats + s * 3 * BM;
 #pragma unroll
       for (int e = 0; e < BM / 32; ++e) {
-        const int rr = lane + 32 * e, r = r0 + rr;
-        const bool in = r < u.q_end;
-        st[rr] = in ? __ldg(b.lse_seg + (size_t)r * p.H + u.head) : 3.0e38f;
-        st[BM + rr] = in ? __ldg(b.dd_seg + (size_t)r * p.H + u.head) : 0.f;
-        st[2 * BM + rr] = in ? __ldg(b.c_seg + r) : 0.f;
+        st[lane + 32 * e] = pre[0][e];
+        st[BM + lane + 32 * e] = pre[1][e];
+        st[2 * BM + lane + 32 * e] = pre[2][e];
       }
       __syncwarp();
       if (lane == 0) {
@@ -370,6 +435,7 @@ bwd_dkdv_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUt
         load_tile<HD>(sbase + SM::kStageB + s * SM::kTile, &tm_do, u.head, r0, bar(BB_FULL + s));
         last[s] = i;
       }
+      fetch(i + 1);
     }
     if (lane == 0) {
       mbar_drain(bar(BB_RES), 0, timeout);
@@ -380,20 +446,34 @@ bwd_dkdv_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUt
   } else if (warp == 5) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      bool ok = mbar_wait(bar(BB_RES), 0, abort_flag, timeout);
-      for (int i = 0; i < n_q && ok; ++i) {
-        const int s = i & 1;
-        if (!(ok = mbar_wait(bar(BB_FULL + s), (i >> 1) & 1, abort_flag, timeout))) break;
+      // 64-query half tiles hq = 2i + h; half hq uses TMEM buffer hq & 1
+      // (S^T at +0, dP^T at +64).  Order: S/dP of hq + 2 right after dV/dK of
+      // hq, so the compute of hq + 1 overlaps those products.
+      const int nh = 2 * n_q;
+      auto issue_sd = [&](int hq) -> bool {
+        const int i = hq >> 1, s = i & 1, h = hq & 1;
+        if (h == 0 && !mbar_wait(bar(BB_FULL + s), (i >> 1) & 1, abort_flag, timeout)) return false;
         tc_fence_after();
         const uint32_t qa = sbase + SM::kStageA + s * SM::kTile, doa = sbase + SM::kStageB + s * SM::kTile;
-        mma_nt<HD>(tmem, sbase + SM::kRes0, qa);          // S^T = K Q^T
-        mma_nt<HD>(tmem + 128, sbase + SM::kRes1, doa);   // dP^T = V dO^T
-        tc_commit(bar(BB_S));
-        if (!(ok = mbar_wait(bar(BB_P), i & 1, abort_flag, timeout))) break;
+        const uint32_t buf = tmem + (hq & 1) * 128;
+        mma_nt_half<HD>(buf, sbase + SM::kRes0, qa, h);        // S^T = K Q^T (64 queries)
+        mma_nt_half<HD>(buf + 64, sbase + SM::kRes1, doa, h);  // dP^T = V dO^T
+        tc_commit(bar(BB_S + (hq & 1)));
+        return true;
+      };
+      bool ok = mbar_wait(bar(BB_RES), 0, abort_flag, timeout);
+      if (ok && nh > 0) ok = issue_sd(0);
+      if (ok && nh > 1) ok = issue_sd(1);
+      for (int hq = 0; hq < nh && ok; ++hq) {
+        const int i = hq >> 1, s = i & 1, h = hq & 1;
+        if (!(ok = mbar_wait(bar(BB_P + (hq & 1)), (hq >> 1) & 1, abort_flag, timeout))) break;
         tc_fence_after();
-        mma_tn<HD>(tmem + 256, tmem, doa, i > 0);             // dV += (c P)^T dO
-        mma_tn<HD>(tmem + 256 + HD, tmem + 128, qa, i > 0);   // dK += dS^T Q
-        tc_commit(bar(BB_EMPTY + s));
+        const uint32_t qa = sbase + SM::kStageA + s * SM::kTile, doa = sbase + SM::kStageB + s * SM::kTile;
+        const uint32_t buf = tmem + (hq & 1) * 128;
+        mma_tn_half<HD>(tmem + 256, buf, doa, h, hq > 0);             // dV += (c P)^T dO
+        mma_tn_half<HD>(tmem + 256 + HD, buf + 64, qa, h, hq > 0);    // dK += dS^T Q
+        if (h == 1) tc_commit(bar(BB_EMPTY + s));   // Q_i, dO_i read by both halves
+        if (hq + 2 < nh) ok = issue_sd(hq + 2);
       }
       tc_commit(bar(BB_DONE));
       tc_commit(bar(BB_END));
@@ -405,43 +485,50 @@ bwd_dkdv_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUt
     // thread = key row of the tile = TMEM lane
     const int row = warp * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
-    const uint32_t s_addr = tmem + lane_addr, dp_addr = tmem + lane_addr + 128;
+    const uint32_t s_addr = tmem + lane_addr;
     const float sl = p.scale_log2, sc = b.scale;
     bool ok = true;
-    for (int i = 0; i < n_q; ++i) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(BB_S), i & 1, abort_flag, timeout));
+    for (int hq = 0; hq < 2 * n_q && ok; ++hq) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(BB_S + (hq & 1)), (hq >> 1) & 1, abort_flag, timeout));
       if (!ok) break;
       tc_fence_after();
-      const float* st = stats + (i & 1) * 3 * BM;
-#pragma unroll 1
-      for (int cc = 0; cc < BM / 32; ++cc) {
-        float sv[32], dpv[32];
-        tmem_ld32(s_addr + cc * 32, sv);
-        tmem_ld32(dp_addr + cc * 32, dpv);
-        tmem_wait_ld();
-        uint32_t pk[16], dk[16];
+      // statistics of the 64 queries of this half (lse, D', c at +0, +BM, +2BM)
+      const float* st = stats + ((hq >> 1) & 1) * 3 * BM + (hq & 1) * (BM / 2);
+      const uint32_t sb = s_addr + (hq & 1) * 128, db = sb + 64;
+      // all 64 scores and dP values of the half with one wait
+      float sv[64], dpv[64];
+      tmem_ld32(sb, sv);
+      tmem_ld32(sb + 32, sv + 32);
+      tmem_ld32(db, dpv);
+      tmem_ld32(db + 32, dpv + 32);
+      tmem_wait_ld();
+      const float4* st4 = reinterpret_cast<const float4*>(st);   // lse, D', c: 4 queries per load
+      float pk[32], dk[32];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float pc[2], ds[2];
+      for (int e4 = 0; e4 < 16; ++e4) {
+        const float4 l4 = st4[e4], d4 = st4[BM / 4 + e4], c4 = st4[BM / 2 + e4];
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w},
+                    cv[4] = {c4.x, c4.y, c4.z, c4.w};
+        float pc[4], ds[4];
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int qi = cc * 32 + 2 * e + h2;
-            const float pr = fast_exp2(sv[2 * e + h2] * sl - st[qi]);
-            const float c = st[2 * BM + qi];
-            pc[h2] = pr * c;
-            ds[h2] = pr * (dpv[2 * e + h2] - st[BM + qi]) * c * sc;
-          }
-          pk[e] = bwd_pack(pc[0], pc[1]);
-          dk[e] = bwd_pack(ds[0], ds[1]);
+        for (int e = 0; e < 4; ++e) {
+          const int qi = 4 * e4 + e;
+          const float pr = fast_exp2(sv[qi] * sl - lv[e]);
+          pc[e] = pr * cv[e];
+          ds[e] = pr * (dpv[qi] - dv4[e]) * cv[e] * sc;
         }
-        // bf16 pairs of 32 queries into columns [16cc, 16cc+16) of each region,
-        // whose fp32 values were read by an earlier chunk (or this one)
-        tmem_st16(s_addr + cc * 16, pk);
-        tmem_st16(dp_addr + cc * 16, dk);
+        pk[2 * e4] = __uint_as_float(bwd_pack(pc[0], pc[1]));
+        pk[2 * e4 + 1] = __uint_as_float(bwd_pack(pc[2], pc[3]));
+        dk[2 * e4] = __uint_as_float(bwd_pack(ds[0], ds[1]));
+        dk[2 * e4 + 1] = __uint_as_float(bwd_pack(ds[2], ds[3]));
       }
+      // bf16 pairs of the 64 queries into the first 32 columns of each half
+      // region (all of whose fp32 values were read above)
+      tmem_st32(sb, pk);
+      tmem_st32(db, dk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(BB_P));
+      mbar_arrive(bar(BB_P + (hq & 1)));
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(BB_DONE), 0, abort_flag, timeout));
     if (ok) {
@@ -464,8 +551,10 @@ bwd_dkdv_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUt
 
 // ------------------------------------------------------------------ dQ
 
-// TMEM: S [0,128) (dS overwrites its first 64 columns), dP [128,256),
-// dQ [256, 256+HD).
+// TMEM: dQ [0, HD), Q [HD, 1.5 HD) and dO [1.5 HD, 2 HD) as bf16 pairs (the
+// A operands of S = Q K^T and dP = dO V^T, so only the streamed K and V
+// halves are read from shared memory), and two 128-column buffers for the
+// 64-key halves (S at +0, dP at +64; dS overwrites the first 32 columns of S).
 template <int HD>
 __global__ void __launch_bounds__(192, 1)
 bwd_dq_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUtensorMap tm_q,
@@ -509,19 +598,31 @@ bwd_dq_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUten
   } else if (warp == 5) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      bool ok = mbar_wait(bar(BB_RES), 0, abort_flag, timeout);
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int s = j & 1;
-        if (!(ok = mbar_wait(bar(BB_FULL + s), (j >> 1) & 1, abort_flag, timeout))) break;
+      // 64-key half tiles hk = 2j + h; half hk uses TMEM buffer hk & 1 (S at
+      // +0, dP at +64); S/dP of hk + 2 right after dQ of hk
+      const int nh = 2 * n_kv;
+      auto issue_sd = [&](int hk) -> bool {
+        const int j = hk >> 1, s = j & 1, h = hk & 1;
+        if (h == 0 && !mbar_wait(bar(BB_FULL + s), (j >> 1) & 1, abort_flag, timeout)) return false;
         tc_fence_after();
         const uint32_t ka = sbase + SM::kStageA + s * SM::kTile, va = sbase + SM::kStageB + s * SM::kTile;
-        mma_nt<HD>(tmem, sbase + SM::kRes0, ka);          // S = Q K^T
-        mma_nt<HD>(tmem + 128, sbase + SM::kRes1, va);    // dP = dO V^T
-        tc_commit(bar(BB_S));
-        if (!(ok = mbar_wait(bar(BB_P), j & 1, abort_flag, timeout))) break;
+        const uint32_t buf = tmem + 2 * HD + (hk & 1) * 128;
+        mma_ts_half<HD>(buf, tmem + HD, ka, h);                // S = Q K^T (64 keys)
+        mma_ts_half<HD>(buf + 64, tmem + HD + HD / 2, va, h);  // dP = dO V^T
+        tc_commit(bar(BB_S + (hk & 1)));
+        return true;
+      };
+      bool ok = mbar_wait(bar(BB_A), 0, abort_flag, timeout);
+      if (ok && nh > 0) ok = issue_sd(0);
+      if (ok && nh > 1) ok = issue_sd(1);
+      for (int hk = 0; hk < nh && ok; ++hk) {
+        const int j = hk >> 1, s = j & 1, h = hk & 1;
+        if (!(ok = mbar_wait(bar(BB_P + (hk & 1)), (hk >> 1) & 1, abort_flag, timeout))) break;
         tc_fence_after();
-        mma_tn<HD>(tmem + 256, tmem, ka, j > 0);          // dQ += dS K
-        tc_commit(bar(BB_EMPTY + s));
+        const uint32_t ka = sbase + SM::kStageA + s * SM::kTile;
+        mma_tn_half<HD>(tmem, tmem + 2 * HD + (hk & 1) * 128, ka, h, hk > 0);   // dQ += dS K
+        if (h == 1) tc_commit(bar(BB_EMPTY + s));
+        if (hk + 2 < nh) ok = issue_sd(hk + 2);
       }
       tc_commit(bar(BB_DONE));
       tc_commit(bar(BB_END));
@@ -533,49 +634,57 @@ bwd_dq_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUten
     // thread = query row of the tile = TMEM lane
     const int row = warp * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
-    const uint32_t s_addr = tmem + lane_addr, dp_addr = tmem + lane_addr + 128;
+    const uint32_t s_addr = tmem + lane_addr;
     const float sl = p.scale_log2;
     const int qr = u.t_begin + row;
     const bool in = qr < u.t_end;
     const float lse = in ? __ldg(b.lse_seg + (size_t)qr * p.H + u.head) : 3.0e38f;
     const float dd = in ? __ldg(b.dd_seg + (size_t)qr * p.H + u.head) : 0.f;
     const float cs = in ? __ldg(b.c_seg + qr) * b.scale : 0.f;
-    bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(BB_S), j & 1, abort_flag, timeout));
-      if (!ok) break;
-      tc_fence_after();
-      const int valid = u.kv_end - (u.kv_begin + j * BN);   // keys of this tile in the segment
-#pragma unroll 1
-      for (int cc = 0; cc < BN / 32; ++cc) {
-        float sv[32], dpv[32];
-        tmem_ld32(s_addr + cc * 32, sv);
-        tmem_ld32(dp_addr + cc * 32, dpv);
-        tmem_wait_ld();
-        uint32_t dk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float ds[2];
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int ki = cc * 32 + 2 * e + h2;
-            const float pr = ki < valid ? fast_exp2(sv[2 * e + h2] * sl - lse) : 0.f;
-            ds[h2] = pr * (dpv[2 * e + h2] - dd) * cs;
-          }
-          dk[e] = bwd_pack(ds[0], ds[1]);
-        }
-        tmem_st16(s_addr + cc * 16, dk);
-      }
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar(BB_RES), 0, abort_flag, timeout));
+    if (ok) {
+      tile_row_to_tmem<HD>(smem + SM::kRes0, row, tmem + lane_addr + HD);            // Q
+      tile_row_to_tmem<HD>(smem + SM::kRes1, row, tmem + lane_addr + HD + HD / 2);   // dO
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(BB_P));
+      mbar_arrive(bar(BB_A));
+    }
+    for (int hk = 0; hk < 2 * n_kv && ok; ++hk) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(BB_S + (hk & 1)), (hk >> 1) & 1, abort_flag, timeout));
+      if (!ok) break;
+      tc_fence_after();
+      // keys of this half tile that belong to the segment
+      const int valid = u.kv_end - (u.kv_begin + (hk >> 1) * BN + (hk & 1) * (BN / 2));
+      const uint32_t sb = s_addr + 2 * HD + (hk & 1) * 128, db = sb + 64;
+      float sv[64], dpv[64];
+      tmem_ld32(sb, sv);
+      tmem_ld32(sb + 32, sv + 32);
+      tmem_ld32(db, dpv);
+      tmem_ld32(db + 32, dpv + 32);
+      tmem_wait_ld();
+      float dk[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        float ds[2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int ki = 2 * e + h2;
+          const float pr = fast_exp2(sv[ki] * sl - lse);
+          ds[h2] = ki < valid ? pr * (dpv[ki] - dd) * cs : 0.f;
+        }
+        dk[e] = __uint_as_float(bwd_pack(ds[0], ds[1]));
+      }
+      tmem_st32(sb, dk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(BB_P + (hk & 1)));
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(BB_DONE), 0, abort_flag, timeout));
     if (ok) {
       tc_fence_after();
       float g[HD];
 #pragma unroll
-      for (int cc = 0; cc < HD / 32; ++cc) tmem_ld32(tmem + lane_addr + 256 + cc * 32, g + cc * 32);
+      for (int cc = 0; cc < HD / 32; ++cc) tmem_ld32(tmem + lane_addr + cc * 32, g + cc * 32);
       tmem_wait_ld();
       if (in) add_rows<HD>(b.dq, token_of(p, qr), p.H, u.head, g);
     }
