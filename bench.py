@@ -534,11 +534,15 @@ def run_train(args):
     # and the recomputed S; the dQ pass recomputes S and dP once more on top of that)
     bwd_moga_tf = 2.5 * fl_fwd_moga / (call_ms["moga_group_attn_bwd"] * 1e-3) / 1e12
     bwd_stga_tf = 2.5 * fl_fwd_stga / (call_ms["stga_attn_bwd"] * 1e-3) / 1e12
+    route_bwd_bytes = N * d * (2 + 4)
     line = {
         "metric": "visual-attn layer training step (fwd + bwd) tokens/s (bf16)", "value": N / (step_ms * 1e-3),
         "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
         "higher_is_better": True, "dtype": "bf16", "data": "synthetic (seeded counter-based generator; no dataset)",
         "config": config_dict(wl), "breakdown_ms": call_ms,
+        "route_bwd_hbm": {"bytes": route_bwd_bytes, "gbs": route_bwd_bytes / (call_ms["moga_route_bwd"] * 1e-3) / 1e9,
+                          "frac": route_bwd_bytes / (call_ms["moga_route_bwd"] * 1e-3) / 1e9 / pk["hbm_gbs"],
+                          "what": "x read (bf16) + dx written (fp32) over the moga_route_bwd call"},
         "attn_bwd_tflops": {"moga": bwd_moga_tf, "stga": bwd_stga_tf,
                             "moga_frac_of_peak": bwd_moga_tf / pk["bf16_tflops"],
                             "convention": "2.5 x forward FLOPs (4*H*hd*sum n_q*n_kv)"},

@@ -65,6 +65,14 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, long l
   }
 }
 
+// 1-D bulk copy global -> shared memory of this CTA (no multicast), completion
+// counted on an mbarrier.  dst, src and bytes must be multiples of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
 // 3-D tiled TMA load: box {64 columns, 1 head, 128 rows}.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int col, int head, int row,
                                             uint32_t bar) {
