@@ -265,8 +265,9 @@ moga_status stga_attn_bwd(const void* q, const void* k, const void* v, int32_t H
                           const float* o_frame, const float* lse_frame, const void* dout,
                           float* dq, float* dk, float* dv, void* ws, size_t ws_bytes, void* stream);
 
-/* Router backward workspace (per-block partial sums of dW_r); 256-byte
- * aligned.  Returns 0 for arguments moga_route_bwd would reject. */
+/* Router backward workspace (dr per token, per-block partial sums of dW_r
+ * and dbias); 256-byte aligned.  Returns 0 for arguments moga_route_bwd
+ * would reject. */
 size_t moga_route_bwd_ws_bytes(int64_t N, int32_t d, int32_t M);
 
 /* Router backward through the gate and the balancing loss:
@@ -276,7 +277,9 @@ size_t moga_route_bwd_ws_bytes(int64_t N, int32_t d, int32_t M);
  *   dbias = sum_t dr[t] ([M] fp32, written; NULL to skip).
  * x, w_r: as for moga_route (dtype dt);  group_id, probs: from
  * moga_route_train;  dgate: from moga_group_attn_bwd;  counts: from
- * moga_permute;  dloss: the objective's weight on L_gb. */
+ * moga_permute;  dloss: the objective's weight on L_gb.  d must be a
+ * positive multiple of 8 and x, dx 16-byte aligned (MOGA_ERR_INVALID_ARG
+ * otherwise).  Deterministic: every sum runs in a fixed order. */
 moga_status moga_route_bwd(const void* x, const void* w_r, moga_dtype dt, int64_t N, int32_t d, int32_t M,
                            const int32_t* group_id, const float* probs, const float* dgate,
                            const int32_t* counts, float alpha, float dloss,
