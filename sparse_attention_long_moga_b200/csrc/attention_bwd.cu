@@ -9,8 +9,9 @@
 // dS = P * (dP - D),  dQ = dS K * scale,  dK = dS^T Q * scale.
 // The layer's upstream gradient dout reaches each branch through the mean
 // (1/3) and, for MoGA, the gate: dO = c * dout with c = p_g / 3 (MoGA) or
-// 1/3 (static).  c is applied in fp32 inside the kernels (to P for dV and to
-// dS), so the bf16 copy of dout is exact.  D is taken as c * D' with
+// 1/3 (static).  c is applied in fp32 inside the kernels, folded into the
+// exponent (2^(S sl - lse + log2 c) = c P), so the bf16 copy of dout is
+// exact; the softmax scale of dS is applied to dK and dQ in the epilogues.  D is taken as c * D' with
 // D' = rowsum(dout * O_attn); for MoGA O_attn = o_moga / p_g, which also gives
 // the gate's gradient  dgate[t] = sum_h D'[t, h] / 3.
 //
@@ -44,9 +45,8 @@ namespace attn {
 struct BwdParams {
   Params f;               // branch, geometry, perm / cu / gate, N, H, scale_log2
   float scale;            // softmax scale
-  const float* lse_seg;   // [N][H] forward log-sum-exp (log2 domain), segment order
+  const float* lse_seg;   // [N][H] forward log-sum-exp (log2 domain) less log2 c, segment order
   const float* dd_seg;    // [N][H] D' = rowsum(dout * O_attn), segment order
-  const float* c_seg;     // [N] c = gate / 3 (MoGA) or 1 / 3, segment order
   float* dq;              // [N][H][hd] fp32, token order, added to
   float* dk;
   float* dv;
@@ -127,14 +127,15 @@ __device__ __forceinline__ Unit decode_unit(const BwdParams& b, const GroupTable
 
 // One warp per segment position j.  Copies the Q, K, V and dout rows of the
 // token at position j into segment order (not for frames, already in order),
-// and writes lse_seg, dd_seg (D') and c_seg; MoGA also writes dgate.
+// and writes lse_seg (the forward's log-sum-exp less log2 c, so that
+// 2^(S sl - lse_seg) = c P) and dd_seg (D'); MoGA also writes dgate.
 template <int MODE>
 __global__ void __launch_bounds__(256)
 bwd_prep_kernel(const __grid_constant__ BwdParams b, const uint4* __restrict__ q, const uint4* __restrict__ k,
                 const uint4* __restrict__ v, const uint4* __restrict__ dout, const float* __restrict__ o_branch,
                 const float* __restrict__ lse, uint4* __restrict__ qd, uint4* __restrict__ kd, uint4* __restrict__ vd,
                 uint4* __restrict__ dod, float* __restrict__ lse_seg, float* __restrict__ dd_seg,
-                float* __restrict__ c_seg, float* __restrict__ dgate, int hd) {
+                float* __restrict__ dgate, int hd) {
   const Params& p = b.f;
   const int j = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (j >= p.N) return;
@@ -154,6 +155,7 @@ bwd_prep_kernel(const __grid_constant__ BwdParams b, const uint4* __restrict__ q
   // D'[h] = sum_d dout[src][h][d] * o[src][h][d] (/ gate for MoGA): each lane
   // takes 8 consecutive elements; hd / 8 lanes cover one head
   const float gsc = MODE == MODE_MOGA ? __ldg(p.gate + src) : 1.0f;
+  const float log2c = log2f(gsc / 3.0f);   // c = gate / 3 (MoGA) or 1 / 3
   const int lph = hd / 8;              // lanes per head
   const float4* orow = reinterpret_cast<const float4*>(o_branch) + (size_t)src * p.H * hd / 4;
   float dsum = 0.f;
@@ -177,7 +179,7 @@ bwd_prep_kernel(const __grid_constant__ BwdParams b, const uint4* __restrict__ q
       const int h = c / lph;
       const float dd = part / gsc;
       dd_seg[(size_t)j * p.H + h] = dd;
-      lse_seg[(size_t)j * p.H + h] = __ldg(lse + (size_t)src * p.H + h);
+      lse_seg[(size_t)j * p.H + h] = __ldg(lse + (size_t)src * p.H + h) - log2c;
       dsum += dd;
     }
   }
@@ -186,7 +188,6 @@ bwd_prep_kernel(const __grid_constant__ BwdParams b, const uint4* __restrict__ q
     for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
     if (lane == 0) dgate[src] = dsum / 3.0f;
   }
-  if (lane == 0) c_seg[j] = gsc / 3.0f;
 }
 
 // ------------------------------------------------------------------ shared pieces
@@ -218,9 +219,24 @@ enum BwdBar : int {
   BB_DONE = 9,       // accumulators final
   BB_END = 10,       // every MMA finished (teardown)
   BB_A = 11,         // resident operands copied into TMEM (128 arrivals)
-  BB_COUNT = 12
+  BB_STATS = 12,     // +stage: a query tile's statistics landed (dK/dV; 32 cp.async arrivals)
+  BB_COUNT = 14
 };
 static_assert(BB_COUNT <= BwdSmem<128>::kNumBars, "barrier area");
+
+// Statistics of a row past the segment: an exponent offset that makes c P
+// exactly 0, and D' = 0 (source of the cp.async that fills such rows).
+__device__ float g_bwd_stat_pad[2] = {3.0e38f, 0.0f};
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const float* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+// arrive on bar once this thread's earlier cp.async copies have landed (the
+// barrier's count includes the arrival)
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t bwd_pack(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -264,6 +280,7 @@ __device__ __forceinline__ bool bwd_setup(const BwdParams& b, uint8_t* smem, uin
     mbar_init(bar0 + 8 * BB_DONE, 1);
     mbar_init(bar0 + 8 * BB_END, 1);
     mbar_init(bar0 + 8 * BB_A, BM);
+    for (int s = 0; s < 2; ++s) mbar_init(bar0 + 8 * (BB_STATS + s), 32);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -380,7 +397,7 @@ bwd_dkdv_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUt
   const uint32_t sbase = smem_u32(smem);
   auto bar = [&](int i) { return sbase + SM::kBar + 8u * (uint32_t)i; };
   volatile int* abort_flag = reinterpret_cast<int*>(smem + SM::kMisc);
-  float* stats = reinterpret_cast<float*>(smem + SM::kStats);   // [2][3][BM]: lse, D', c
+  float* stats = reinterpret_cast<float*>(smem + SM::kStats);   // [2][2][BM]: lse - log2 c, D'
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long timeout = b.f.timeout_cycles;
   const Params& p = b.f;
@@ -398,45 +415,32 @@ bwd_dkdv_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUt
       load_tile<HD>(sbase + SM::kRes0, &tm_k, u.head, u.t_begin, bar(BB_RES));
       load_tile<HD>(sbase + SM::kRes1, &tm_v, u.head, u.t_begin, bar(BB_RES));
     }
-    // per-query statistics of a tile (lse, D', c for 128 rows, 4 per lane);
-    // rows past the segment get c = 0 and a huge log-sum-exp, so their P and
-    // dS are exactly 0.  Loaded a tile ahead, so the global-load latency
-    // overlaps the wait for the stage.
-    float pre[3][BM / 32];
-    auto fetch = [&](int i) {
-      const int r0 = u.q_begin + i * BM;
-#pragma unroll
-      for (int e = 0; e < BM / 32; ++e) {
-        const int r = r0 + lane + 32 * e;
-        const bool in = i < n_q && r < u.q_end;
-        pre[0][e] = in ? __ldg(b.lse_seg + (size_t)r * p.H + u.head) : 3.0e38f;
-        pre[1][e] = in ? __ldg(b.dd_seg + (size_t)r * p.H + u.head) : 0.f;
-        pre[2][e] = in ? __ldg(b.c_seg + r) : 0.f;
-      }
-    };
-    fetch(0);
     for (int i = 0; i < n_q && ok; ++i) {
       const int s = i & 1;
       const uint32_t ph = (i >> 1) & 1;
       ok = __shfl_sync(0xffffffffu, lane == 0 ? (int)mbar_wait(bar(BB_EMPTY + s), ph ^ 1, abort_flag, timeout) : 0, 0);
       if (!ok) break;
       const int r0 = u.q_begin + i * BM;
-      float* st = stats + s * 3 * BM;
-#pragma unroll
-      for (int e = 0; e < BM / 32; ++e) {
-        st[lane + 32 * e] = pre[0][e];
-        st[BM + lane + 32 * e] = pre[1][e];
-        st[2 * BM + lane + 32 * e] = pre[2][e];
-      }
-      __syncwarp();
       if (lane == 0) {
         mbar_arrive_expect_tx(bar(BB_FULL + s), 2 * SM::kTile);
         load_tile<HD>(sbase + SM::kStageA + s * SM::kTile, &tm_q, u.head, r0, bar(BB_FULL + s));
         load_tile<HD>(sbase + SM::kStageB + s * SM::kTile, &tm_do, u.head, r0, bar(BB_FULL + s));
         last[s] = i;
       }
-      fetch(i + 1);
+      // the tile's per-query statistics (lse - log2 c, D'), 4 rows per lane,
+      // by asynchronous copies that complete on BB_STATS; rows past the
+      // segment copy the pad values, so their c P and dS are exactly 0
+      const uint32_t st = sbase + SM::kStats + (uint32_t)(s * 2 * BM * 4);
+#pragma unroll
+      for (int e = 0; e < BM / 32; ++e) {
+        const int qi = lane + 32 * e, r = r0 + qi;
+        const bool in = r < u.q_end;
+        cp_async4(st + qi * 4, in ? b.lse_seg + (size_t)r * p.H + u.head : &g_bwd_stat_pad[0]);
+        cp_async4(st + (BM + qi) * 4, in ? b.dd_seg + (size_t)r * p.H + u.head : &g_bwd_stat_pad[1]);
+      }
+      cp_async_arrive_noinc(bar(BB_STATS + s));
     }
+    cp_async_wait_all();
     if (lane == 0) {
       mbar_drain(bar(BB_RES), 0, timeout);
       for (int s = 0; s < 2; ++s)
@@ -471,7 +475,7 @@ bwd_dkdv_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUt
         const uint32_t qa = sbase + SM::kStageA + s * SM::kTile, doa = sbase + SM::kStageB + s * SM::kTile;
         const uint32_t buf = tmem + (hq & 1) * 128;
         mma_tn_half<HD>(tmem + 256, buf, doa, h, hq > 0);             // dV += (c P)^T dO
-        mma_tn_half<HD>(tmem + 256 + HD, buf + 64, qa, h, hq > 0);    // dK += dS^T Q
+        mma_tn_half<HD>(tmem + 256 + HD, buf + 64, qa, h, hq > 0);    // dK += dS^T Q / scale
         if (h == 1) tc_commit(bar(BB_EMPTY + s));   // Q_i, dO_i read by both halves
         if (hq + 2 < nh) ok = issue_sd(hq + 2);
       }
@@ -486,14 +490,16 @@ bwd_dkdv_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUt
     const int row = warp * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
     const uint32_t s_addr = tmem + lane_addr;
-    const float sl = p.scale_log2, sc = b.scale;
+    const float sl = p.scale_log2;
     bool ok = true;
     for (int hq = 0; hq < 2 * n_q && ok; ++hq) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(BB_S + (hq & 1)), (hq >> 1) & 1, abort_flag, timeout));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(BB_S + (hq & 1)), (hq >> 1) & 1, abort_flag, timeout) &&
+                                       ((hq & 1) || mbar_wait(bar(BB_STATS + ((hq >> 1) & 1)), (hq >> 2) & 1,
+                                                              abort_flag, timeout)));
       if (!ok) break;
       tc_fence_after();
-      // statistics of the 64 queries of this half (lse, D', c at +0, +BM, +2BM)
-      const float* st = stats + ((hq >> 1) & 1) * 3 * BM + (hq & 1) * (BM / 2);
+      // statistics of the 64 queries of this half (lse - log2 c at +0, D' at +BM)
+      const float* st = stats + ((hq >> 1) & 1) * 2 * BM + (hq & 1) * (BM / 2);
       const uint32_t sb = s_addr + (hq & 1) * 128, db = sb + 64;
       // all 64 scores and dP values of the half with one wait
       float sv[64], dpv[64];
@@ -502,20 +508,18 @@ bwd_dkdv_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUt
       tmem_ld32(db, dpv);
       tmem_ld32(db + 32, dpv + 32);
       tmem_wait_ld();
-      const float4* st4 = reinterpret_cast<const float4*>(st);   // lse, D', c: 4 queries per load
+      const float4* st4 = reinterpret_cast<const float4*>(st);   // 4 queries per load
       float pk[32], dk[32];
 #pragma unroll
       for (int e4 = 0; e4 < 16; ++e4) {
-        const float4 l4 = st4[e4], d4 = st4[BM / 4 + e4], c4 = st4[BM / 2 + e4];
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w},
-                    cv[4] = {c4.x, c4.y, c4.z, c4.w};
+        const float4 l4 = st4[e4], d4 = st4[BM / 4 + e4];
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
         float pc[4], ds[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int qi = 4 * e4 + e;
-          const float pr = fast_exp2(sv[qi] * sl - lv[e]);
-          pc[e] = pr * cv[e];
-          ds[e] = pr * (dpv[qi] - dv4[e]) * cv[e] * sc;
+          pc[e] = fast_exp2(sv[qi] * sl - lv[e]);   // c P
+          ds[e] = pc[e] * (dpv[qi] - dv4[e]);       // dS / scale
         }
         pk[2 * e4] = __uint_as_float(bwd_pack(pc[0], pc[1]));
         pk[2 * e4 + 1] = __uint_as_float(bwd_pack(pc[2], pc[3]));
@@ -542,6 +546,9 @@ bwd_dkdv_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUt
 #pragma unroll
         for (int cc = 0; cc < HD / 32; ++cc) tmem_ld32(tmem + lane_addr + 256 + part * HD + cc * 32, g + cc * 32);
         tmem_wait_ld();
+        if (part == 1)
+#pragma unroll
+          for (int e = 0; e < HD; ++e) g[e] *= b.scale;   // dK = scale dS^T Q
         if (in) add_rows<HD>(part == 0 ? b.dv : b.dk, tok, p.H, u.head, g);
       }
     }
@@ -620,7 +627,7 @@ bwd_dq_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUten
         if (!(ok = mbar_wait(bar(BB_P + (hk & 1)), (hk >> 1) & 1, abort_flag, timeout))) break;
         tc_fence_after();
         const uint32_t ka = sbase + SM::kStageA + s * SM::kTile;
-        mma_tn_half<HD>(tmem, tmem + 2 * HD + (hk & 1) * 128, ka, h, hk > 0);   // dQ += dS K
+        mma_tn_half<HD>(tmem, tmem + 2 * HD + (hk & 1) * 128, ka, h, hk > 0);   // dQ += dS K / scale
         if (h == 1) tc_commit(bar(BB_EMPTY + s));
         if (hk + 2 < nh) ok = issue_sd(hk + 2);
       }
@@ -638,9 +645,9 @@ bwd_dq_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUten
     const float sl = p.scale_log2;
     const int qr = u.t_begin + row;
     const bool in = qr < u.t_end;
-    const float lse = in ? __ldg(b.lse_seg + (size_t)qr * p.H + u.head) : 3.0e38f;
+    // log-sum-exp less log2 c, so 2^(S sl - lse2) is c P; huge past the segment
+    const float lse2 = in ? __ldg(b.lse_seg + (size_t)qr * p.H + u.head) : 3.0e38f;
     const float dd = in ? __ldg(b.dd_seg + (size_t)qr * p.H + u.head) : 0.f;
-    const float cs = in ? __ldg(b.c_seg + qr) * b.scale : 0.f;
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar(BB_RES), 0, abort_flag, timeout));
     if (ok) {
       tile_row_to_tmem<HD>(smem + SM::kRes0, row, tmem + lane_addr + HD);            // Q
@@ -669,8 +676,8 @@ bwd_dq_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUten
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
           const int ki = 2 * e + h2;
-          const float pr = fast_exp2(sv[ki] * sl - lse);
-          ds[h2] = ki < valid ? pr * (dpv[ki] - dd) * cs : 0.f;
+          const float pc = fast_exp2(sv[ki] * sl - lse2);
+          ds[h2] = ki < valid ? pc * (dpv[ki] - dd) : 0.f;   // dS / scale
         }
         dk[e] = __uint_as_float(bwd_pack(ds[0], ds[1]));
       }
@@ -686,6 +693,8 @@ bwd_dq_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUten
 #pragma unroll
       for (int cc = 0; cc < HD / 32; ++cc) tmem_ld32(tmem + lane_addr + cc * 32, g + cc * 32);
       tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < HD; ++e) g[e] *= b.scale;   // dQ = scale dS K
       if (in) add_rows<HD>(b.dq, token_of(p, qr), p.H, u.head, g);
     }
   }
@@ -696,15 +705,15 @@ bwd_dq_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUten
 
 static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// q, k, v, dout in segment order, then lse_seg, dd_seg [N][H], c_seg [N]
+// q, k, v, dout in segment order, then lse_seg, dd_seg [N][H]
 static size_t bwd_ws_bytes(int64_t N, int H, int hd) {
   const size_t t = align256((size_t)N * H * hd * 2);
-  return 4 * t + 2 * align256((size_t)N * H * 4) + align256((size_t)N * 4);
+  return 4 * t + 2 * align256((size_t)N * H * 4);
 }
 
 struct BwdWs {
   uint8_t *q, *k, *v, *dout;
-  float *lse, *dd, *c;
+  float *lse, *dd;
 };
 
 static BwdWs carve_bwd_ws(void* ws, int64_t N, int H, int hd) {
@@ -717,7 +726,6 @@ static BwdWs carve_bwd_ws(void* ws, int64_t N, int H, int hd) {
   r.dout = w + 3 * t;
   r.lse = reinterpret_cast<float*>(w + 4 * t);
   r.dd = reinterpret_cast<float*>(w + 4 * t + st);
-  r.c = reinterpret_cast<float*>(w + 4 * t + 2 * st);
   return r;
 }
 
@@ -754,7 +762,6 @@ static moga_status run_branch_bwd(BwdParams& b, int hd, int q_units, int kv_unit
   const BwdWs w = carve_bwd_ws(ws, b.f.N, b.f.H, hd);
   b.lse_seg = w.lse;
   b.dd_seg = w.dd;
-  b.c_seg = w.c;
   const int grid = ceil_div(b.f.N, 8);
   const uint4 *q4 = static_cast<const uint4*>(q), *k4 = static_cast<const uint4*>(k),
               *v4 = static_cast<const uint4*>(v), *d4 = static_cast<const uint4*>(dout);
@@ -762,13 +769,13 @@ static moga_status run_branch_bwd(BwdParams& b, int hd, int q_units, int kv_unit
         *dd = reinterpret_cast<uint4*>(w.dout);
   if (b.f.mode == MODE_MOGA)
     bwd_prep_kernel<MODE_MOGA><<<grid, 256, 0, s>>>(b, q4, k4, v4, d4, o_branch, lse, qd, kd, vd, dd, w.lse, w.dd,
-                                                     w.c, dgate, hd);
+                                                     dgate, hd);
   else if (b.f.mode == MODE_WINDOW)
     bwd_prep_kernel<MODE_WINDOW><<<grid, 256, 0, s>>>(b, q4, k4, v4, d4, o_branch, lse, qd, kd, vd, dd, w.lse, w.dd,
-                                                       w.c, dgate, hd);
+                                                       dgate, hd);
   else
     bwd_prep_kernel<MODE_FRAME><<<grid, 256, 0, s>>>(b, q4, k4, v4, d4, o_branch, lse, qd, kd, vd, dd, w.lse, w.dd,
-                                                      w.c, dgate, hd);
+                                                      dgate, hd);
   moga_status st = check_launch("attention backward (prep)");
   if (st != MOGA_OK) return st;
   const bool in_place = b.f.mode == MODE_FRAME;
