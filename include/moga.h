@@ -285,6 +285,52 @@ moga_status moga_route_bwd(const void* x, const void* w_r, moga_dtype dt, int64_
                            const int32_t* counts, float alpha, float dloss,
                            float* dx, float* dw_r, float* dbias, void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------- batch of videos --
+ * B videos of n_per tokens each, flattened video-major (token t of video b is
+ * row b * n_per + t), sharing the router (MoGA note, key design 1: routing is
+ * per token; training setup: the MMDiT-based model at M = 20).  Readings: a
+ * token's MoGA group holds tokens of its own video only (sort key
+ * b * M + g(x), so B * M segments), the STGA groups are per video with one
+ * geometry, and L_gb takes F_i and P_i over all B * n_per tokens.  Route the
+ * batch with moga_route(N = B * n_per) and average with visual_attn_mean.
+ */
+
+/* Permute workspace for a batch; 0 for arguments the call would reject. */
+size_t moga_permute_batched_ws_bytes(int64_t n_per, int32_t B, int32_t M);
+
+/* Stable counting sort of B * n_per tokens by b * M + group_id:
+ *   perm:       [B*n_per] int32, flattened token indices, segment-major
+ *   cu_seqlens: [B*M + 1] int32;  counts: [B*M] int32 (segment b*M + i holds
+ *               video b's tokens of group i);  max_seqlen: [1] int32
+ * Requires B * n_per < 2^31, 1 <= M <= 32 and B * M <= 1024
+ * (MOGA_ERR_UNSUPPORTED above).  Bit-identical to moga_permute when B = 1. */
+moga_status moga_permute_batched(const int32_t* group_id, int64_t n_per, int32_t B, int32_t M,
+                                 int32_t* perm, int32_t* cu_seqlens, int32_t* counts,
+                                 int32_t* max_seqlen, void* ws, size_t ws_bytes, void* stream);
+
+/* MoGA attention of a batch: as moga_group_attn over N = B * n_per tokens
+ * with perm / cu_seqlens from moga_permute_batched (video b's groups are
+ * segments [b M, b M + M)); o_acc [B*n_per][H][hd] fp32 written (=);
+ * lse [B*n_per][H] fp32 (log2 domain) written when not NULL.  Workspace:
+ * moga_attn_ws_bytes(B * n_per, H, hd).  One gather, one launch per video. */
+moga_status moga_group_attn_batched(const void* q, const void* k, const void* v, int64_t n_per, int32_t B,
+                                    int32_t H, int32_t hd, const int32_t* perm, const int32_t* cu_seqlens,
+                                    int32_t M, const float* gate_prob, float softmax_scale, float* o_acc,
+                                    float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* STGA of a batch: stga_attn on each video's slice (geometry per video,
+ * N = T*h*w tokens each); o_acc [B*N][H][hd] accumulates (+=).  Workspace:
+ * moga_attn_ws_bytes(N, H, hd) (one video's, reused in stream order). */
+moga_status stga_attn_batched(const void* q, const void* k, const void* v, int32_t B, int32_t H, int32_t hd,
+                              const moga_stga_geom* geom, float softmax_scale, float* o_acc, void* ws,
+                              size_t ws_bytes, void* stream);
+
+/* L_gb of a batch: counts [B*M] from moga_permute_batched (summed over the
+ * videos per group), route_ws from moga_route over the N = B * n_per tokens;
+ * N must be a multiple of B.  loss: [1] double, written. */
+moga_status moga_balance_loss_batched(const int32_t* counts, int32_t B, const void* route_ws, int64_t N,
+                                      int32_t M, float alpha, double* loss, void* stream);
+
 /* ------------------------------------------------------------- diagnostics */
 /* Text of the last host-side error of the calling thread ("" if none). */
 const char* moga_last_error(void);

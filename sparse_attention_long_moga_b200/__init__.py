@@ -208,6 +208,65 @@ def visual_attention_forward(x, w_r, bias, q, k, v, M: int, geom: dict, alpha: f
     return dict(out=out, loss=loss, g=g, gate=gate, perm=perm, cu_seqlens=cu, counts=counts, max_seqlen=mx)
 
 
+# ---------------------------------------------------------------- batch
+#
+# B videos of the same shape, video-major: x [B, N, d], q/k/v [B, N, H, hd].
+# The router is shared; a token's MoGA group holds tokens of its own video
+# (segments b * M + g), the STGA groups are per video, and L_gb is taken over
+# the whole batch.
+
+def moga_permute_batched(group_id: torch.Tensor, B: int, M: int):
+    """Stable permute by b * M + g of B * n_per flattened tokens.  Returns
+    (perm [B*n_per], cu_seqlens [B*M+1], counts [B*M], max_seqlen [1]), int32."""
+    _need(group_id, torch.int32, "group_id", 1)
+    n = group_id.shape[0]
+    if B < 1 or n % B:
+        raise ValueError("group_id length %d is not a multiple of B=%d" % (n, B))
+    L = lib()
+    ws_bytes = L.moga_permute_batched_ws_bytes(n // B, B, M)
+    if ws_bytes == 0:
+        raise ValueError("unsupported batch: B=%d, M=%d, n_per=%d" % (B, M, n // B))
+    dev = group_id.device
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    perm = torch.empty(n, dtype=torch.int32, device=dev)
+    cu = torch.empty(B * M + 1, dtype=torch.int32, device=dev)
+    counts = torch.empty(B * M, dtype=torch.int32, device=dev)
+    mx = torch.empty(1, dtype=torch.int32, device=dev)
+    check(L.moga_permute_batched(_ptr(group_id), n // B, B, M, _ptr(perm), _ptr(cu), _ptr(counts), _ptr(mx),
+                                 _ptr(ws), ws.numel(), _stream()), "moga_permute_batched")
+    return perm, cu, counts, mx
+
+
+def visual_attention_forward_batched(x, w_r, bias, q, k, v, M: int, geom: dict, alpha: float,
+                                     softmax_scale: float | None = None):
+    """The layer over a batch of B videos: x [B, N, d], q/k/v [B, N, H, hd] bf16.
+    Returns dict(out bf16 [B, N, H, hd], loss fp64 [1], g, gate, perm, cu_seqlens, counts)."""
+    if x.dim() != 3 or q.dim() != 4:
+        raise ValueError("x must be [B, N, d] and q, k, v [B, N, H, hd]")
+    B, N, d = x.shape
+    if q.shape[:2] != (B, N) or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must be [B, N, H, hd] with x's B and N")
+    H, hd = q.shape[2], q.shape[3]
+    qf, kf, vf = (t.reshape(B * N, H, hd) for t in (q, k, v))
+    g, gate, rws = moga_route(x.reshape(B * N, d), w_r, bias)
+    perm, cu, counts, mx = moga_permute_batched(g, B, M)
+    L = lib()
+    scale = 1.0 / math.sqrt(hd) if softmax_scale is None else softmax_scale
+    ws = attn_workspace(qf)
+    o = torch.empty((B * N, H, hd), dtype=torch.float32, device=q.device)
+    check(L.moga_group_attn_batched(_ptr(qf), _ptr(kf), _ptr(vf), N, B, H, hd, _ptr(perm), _ptr(cu), M, _ptr(gate),
+                                    scale, _ptr(o), None, _ptr(ws), ws.numel(), _stream()), "moga_group_attn_batched")
+    s, keep = geom_struct(geom)
+    check(L.stga_attn_batched(_ptr(qf), _ptr(kf), _ptr(vf), B, H, hd, ctypes.byref(s), scale, _ptr(o), _ptr(ws),
+                              ws.numel(), _stream()), "stga_attn_batched")
+    del keep
+    out = visual_attn_mean(o).reshape(B, N, H, hd)
+    loss = torch.empty(1, dtype=torch.float64, device=x.device)
+    check(L.moga_balance_loss_batched(_ptr(counts), B, _ptr(rws), B * N, M, alpha, _ptr(loss), _stream()),
+          "moga_balance_loss_batched")
+    return dict(out=out, loss=loss, g=g, gate=gate, perm=perm, cu_seqlens=cu, counts=counts, max_seqlen=mx)
+
+
 # ---------------------------------------------------------------- training
 #
 # The training forward keeps the router probabilities, the three branch

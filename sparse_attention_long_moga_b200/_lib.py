@@ -32,6 +32,12 @@ SIGNATURES = {
     "stga_attn_mean": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _P, _F32, _P, _P, _P, _SZ, _P]),
     "visual_attn_mean": (ctypes.c_int, [_P, _I64, _P, _P]),
     "moga_balance_loss": (ctypes.c_int, [_P, _P, _I64, _I32, _F32, _P, _P]),
+    "moga_permute_batched_ws_bytes": (_SZ, [_I64, _I32, _I32]),
+    "moga_permute_batched": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moga_group_attn_batched": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I32, _I32, _P, _P, _I32, _P, _F32, _P, _P,
+                                               _P, _SZ, _P]),
+    "stga_attn_batched": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _P, _F32, _P, _P, _SZ, _P]),
+    "moga_balance_loss_batched": (ctypes.c_int, [_P, _I32, _P, _I64, _I32, _F32, _P, _P]),
     "moga_route_train": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _I64, _I32, _I32, _P, _P, _P, _P, _SZ, _P]),
     "moga_group_attn_train": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I32, _P, _P, _I32, _P, _F32, _P, _P, _P, _SZ,
                                              _P]),

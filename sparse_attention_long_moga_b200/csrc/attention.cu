@@ -785,10 +785,13 @@ extern "C" size_t moga_attn_ws_bytes(int64_t N, int32_t H, int32_t hd) {
   return attn_ws_bytes(N, H, hd);
 }
 
-static moga_status moga_impl(const void* q, const void* k, const void* v, int64_t N, int32_t H, int32_t hd,
-                             const int32_t* perm, const int32_t* cu_seqlens, int32_t M, const float* gate_prob,
-                             float softmax_scale, float* o_acc, float* lse, void* ws, size_t ws_bytes,
-                             void* stream) {
+// B videos of N / B tokens each (B = 1: one video): cu_seqlens holds B * M + 1
+// boundaries, video b's groups are segments [b M, b M + M).  One gather into
+// segment order, then one attention launch per video.
+static moga_status moga_impl(const void* q, const void* k, const void* v, int64_t N, int32_t B, int32_t H,
+                             int32_t hd, const int32_t* perm, const int32_t* cu_seqlens, int32_t M,
+                             const float* gate_prob, float softmax_scale, float* o_acc, float* lse, void* ws,
+                             size_t ws_bytes, void* stream) {
   moga_status st = check_common(q, k, v, N, H, hd, o_acc, ws, ws_bytes, true, "moga_group_attn");
   if (st != MOGA_OK) return st;
   if (!perm || !cu_seqlens || !gate_prob) return fail(MOGA_ERR_INVALID_ARG, "moga_group_attn: null pointer");
@@ -811,17 +814,31 @@ static moga_status moga_impl(const void* q, const void* k, const void* v, int64_
   if ((st = launch_gather(prm, hd, q, k, v, ws, s)) != MOGA_OK) return st;
   const uint8_t* w = static_cast<const uint8_t*>(ws);
   const size_t bytes = (size_t)N * H * hd * 2;
-  // upper bound on the tile count: sum_i ceil(n_i / 256) <= N / 256 + M
-  const int tiles = (ceil_div((int)N, 2 * BM) + M) * H;
-  return dispatch_attn(prm, tiles, hd, w, w + bytes, w + 2 * bytes, s);
+  // upper bound on a video's tile count: sum_i ceil(n_i / 256) <= n / 256 + M
+  const int tiles = (ceil_div((int)(N / B), 2 * BM) + M) * H;
+  for (int b = 0; b < B; ++b) {
+    prm.cu = cu_seqlens + (size_t)b * M;
+    if ((st = dispatch_attn(prm, tiles, hd, w, w + bytes, w + 2 * bytes, s)) != MOGA_OK) return st;
+  }
+  return MOGA_OK;
 }
 
 extern "C" moga_status moga_group_attn(const void* q, const void* k, const void* v, int64_t N, int32_t H, int32_t hd,
                                        const int32_t* perm, const int32_t* cu_seqlens, int32_t M,
                                        const float* gate_prob, float softmax_scale, float* o_acc, void* ws,
                                        size_t ws_bytes, void* stream) {
-  return moga_impl(q, k, v, N, H, hd, perm, cu_seqlens, M, gate_prob, softmax_scale, o_acc, nullptr, ws, ws_bytes,
+  return moga_impl(q, k, v, N, 1, H, hd, perm, cu_seqlens, M, gate_prob, softmax_scale, o_acc, nullptr, ws, ws_bytes,
                    stream);
+}
+
+extern "C" moga_status moga_group_attn_batched(const void* q, const void* k, const void* v, int64_t n_per, int32_t B,
+                                               int32_t H, int32_t hd, const int32_t* perm, const int32_t* cu_seqlens,
+                                               int32_t M, const float* gate_prob, float softmax_scale, float* o_acc,
+                                               float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (B < 1 || n_per <= 0 || n_per * B > INT32_MAX)
+    return fail(MOGA_ERR_INVALID_ARG, "moga_group_attn_batched: B=%d x n_per=%lld out of range", B, (long long)n_per);
+  return moga_impl(q, k, v, n_per * B, B, H, hd, perm, cu_seqlens, M, gate_prob, softmax_scale, o_acc, lse, ws,
+                   ws_bytes, stream);
 }
 
 extern "C" moga_status moga_group_attn_train(const void* q, const void* k, const void* v, int64_t N, int32_t H,
@@ -829,7 +846,7 @@ extern "C" moga_status moga_group_attn_train(const void* q, const void* k, const
                                              const float* gate_prob, float softmax_scale, float* o_moga, float* lse,
                                              void* ws, size_t ws_bytes, void* stream) {
   if (!lse) return fail(MOGA_ERR_INVALID_ARG, "moga_group_attn_train: null lse");
-  return moga_impl(q, k, v, N, H, hd, perm, cu_seqlens, M, gate_prob, softmax_scale, o_moga, lse, ws, ws_bytes,
+  return moga_impl(q, k, v, N, 1, H, hd, perm, cu_seqlens, M, gate_prob, softmax_scale, o_moga, lse, ws, ws_bytes,
                    stream);
 }
 
@@ -919,6 +936,27 @@ extern "C" moga_status stga_attn(const void* q, const void* k, const void* v, in
                                  size_t ws_bytes, void* stream) {
   return stga_impl(q, k, v, H, hd, geom, softmax_scale, o_acc, o_acc, nullptr, nullptr, false, nullptr, ws, ws_bytes,
                    stream, "stga_attn");
+}
+
+// B videos of the same geometry, video-major: one pair of launches per video
+// on its slice of q, k, v and o_acc (the workspace is reused in stream order).
+extern "C" moga_status stga_attn_batched(const void* q, const void* k, const void* v, int32_t B, int32_t H, int32_t hd,
+                                         const moga_stga_geom* geom, float softmax_scale, float* o_acc, void* ws,
+                                         size_t ws_bytes, void* stream) {
+  if (B < 1) return fail(MOGA_ERR_INVALID_ARG, "stga_attn_batched: B=%d", B);
+  if (!geom) return fail(MOGA_ERR_INVALID_ARG, "stga_attn_batched: null geometry");
+  const int64_t n = (int64_t)geom->T * geom->h * geom->w;
+  if (n * B * (int64_t)H >= INT32_MAX) return fail(MOGA_ERR_INVALID_ARG, "stga_attn_batched: B*N*H out of range");
+  const size_t elems = (size_t)n * H * hd;
+  for (int b = 0; b < B; ++b) {
+    const size_t off = (size_t)b * elems * 2;
+    moga_status st = stga_impl(static_cast<const uint8_t*>(q) + off, static_cast<const uint8_t*>(k) + off,
+                               static_cast<const uint8_t*>(v) + off, H, hd, geom, softmax_scale, o_acc + b * elems,
+                               o_acc + b * elems, nullptr, nullptr, false, nullptr, ws, ws_bytes, stream,
+                               "stga_attn_batched");
+    if (st != MOGA_OK) return st;
+  }
+  return MOGA_OK;
 }
 
 extern "C" moga_status stga_attn_mean(const void* q, const void* k, const void* v, int32_t H, int32_t hd,

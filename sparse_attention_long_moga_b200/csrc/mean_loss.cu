@@ -44,7 +44,7 @@ __global__ void mean3_tail_kernel(const float* __restrict__ acc, __nv_bfloat16* 
 // does not depend on scheduling.
 __global__ void __launch_bounds__(1024)
 balance_loss_kernel(const int32_t* __restrict__ counts, const float* __restrict__ partial, int rows, int N,
-                    int M, float alpha, double* __restrict__ loss) {
+                    int M, int B, float alpha, double* __restrict__ loss) {
   __shared__ double part[1024];
   __shared__ double slice[32][32];
   const int t = threadIdx.x;
@@ -77,7 +77,9 @@ balance_loss_kernel(const int32_t* __restrict__ counts, const float* __restrict_
     if (t < M) {
       double tot = 0.0;
       for (int jj = 0; jj < 32; ++jj) tot += slice[jj][t];
-      fp = ((double)counts[t] / (double)N) * (tot / (double)N);
+      int cnt = 0;   // tokens of group t over the B videos of a batch
+      for (int b = 0; b < B; ++b) cnt += counts[b * M + t];
+      fp = ((double)cnt / (double)N) * (tot / (double)N);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) fp += __shfl_xor_sync(0xffffffffu, fp, off);
@@ -159,6 +161,18 @@ extern "C" moga_status moga_balance_loss(const int32_t* counts, const void* rout
   if (N <= 0 || N > INT32_MAX) return fail(MOGA_ERR_INVALID_ARG, "moga_balance_loss: N=%lld out of range", (long long)N);
   if (M < 1 || M > 32) return fail(MOGA_ERR_INVALID_ARG, "moga_balance_loss: M=%d not in [1, 32]", M);
   mean_detail::balance_loss_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(
-      counts, static_cast<const float*>(route_ws), route_partial_rows(N), (int)N, M, alpha, loss);
+      counts, static_cast<const float*>(route_ws), route_partial_rows(N), (int)N, M, 1, alpha, loss);
   return check_launch("moga_balance_loss");
+}
+
+extern "C" moga_status moga_balance_loss_batched(const int32_t* counts, int32_t B, const void* route_ws,
+                                                 int64_t N, int32_t M, float alpha, double* loss, void* stream) {
+  using namespace moga;
+  if (!counts || !route_ws || !loss) return fail(MOGA_ERR_INVALID_ARG, "moga_balance_loss_batched: null pointer");
+  if (N <= 0 || N > INT32_MAX || B < 1 || N % B != 0)
+    return fail(MOGA_ERR_INVALID_ARG, "moga_balance_loss_batched: N=%lld, B=%d", (long long)N, B);
+  if (M < 1 || M > 32) return fail(MOGA_ERR_INVALID_ARG, "moga_balance_loss_batched: M=%d not in [1, 32]", M);
+  mean_detail::balance_loss_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(
+      counts, static_cast<const float*>(route_ws), route_partial_rows(N), (int)N, M, B, alpha, loss);
+  return check_launch("moga_balance_loss_batched");
 }

@@ -80,15 +80,6 @@ extern "C" moga_status moga_permute_noalloc(const int32_t* group_id, int64_t N, 
   int32_t* scratch = nullptr;
   moga_status st = scratch_for_current_device(&scratch);
   if (st != MOGA_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int n = (int)N;
-  const int tiles = ceil_div(n, kTile);
-  int32_t* hist = scratch;
-  int32_t* tile_off = scratch + (size_t)tiles * M;
-  tile_hist_kernel<<<tiles, kThreads, 0, s>>>(group_id, n, M, hist);
-  if ((st = check_launch("moga_permute_noalloc/hist")) != MOGA_OK) return st;
-  scan_kernel<<<1, 1024, 0, s>>>(hist, tiles, M, tile_off, cu_seqlens, counts, max_seqlen);
-  if ((st = check_launch("moga_permute_noalloc/scan")) != MOGA_OK) return st;
-  scatter_kernel<<<tiles, kThreads, 0, s>>>(group_id, n, M, tile_off, perm);
-  return check_launch("moga_permute_noalloc/scatter");
+  return run_permute<32>(group_id, (int)N, M, (int)N, M, perm, cu_seqlens, counts, max_seqlen, scratch,
+                         static_cast<cudaStream_t>(stream));
 }
