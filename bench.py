@@ -553,6 +553,94 @@ def run_train(args):
     return 0
 
 
+def run_batch(args):
+    """Forward over a batch of B videos of the 5 s Wan-1.3B shape at M = 20 (the
+    pages' MMDiT group count), per-video groups: route over the B*N tokens,
+    batched permute (B*M segments), batched MoGA, batched STGA, mean and the
+    batch loss, through the C ABI with persistent buffers.  One JSON line
+    (not the headline line)."""
+    import torch
+
+    import sparse_attention_long_moga_b200 as moga
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    B = args.batch
+    per = WORKLOAD.with_(M=20)
+    big = per.with_(name="%s_x%d" % (per.name, B), T=per.T * B, shots=tuple(per.shots) * B)
+    inp = make_inputs(big)
+    geom = W.stga_shape(per)
+
+    def to_dev(a):
+        t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+        return t.to(dev).view(torch.bfloat16) if a.dtype == np.uint16 else t.to(dev)
+
+    x, w_r, q, k, v = (to_dev(inp[n]) for n in ("x", "w_r", "q", "k", "v"))
+    n, M, H, hd, d = per.N, per.M, per.H, per.hd, per.d
+    N = B * n
+    L = moga._lib.lib()
+    sp = moga._stream()
+    P = moga._ptr
+    i32 = dict(dtype=torch.int32, device=dev)
+    g, perm, counts, mx, cu = (torch.empty(c, **i32) for c in (N, N, B * M, 1, B * M + 1))
+    gate = torch.empty(N, dtype=torch.float32, device=dev)
+    rws = torch.empty(max(L.moga_route_ws_bytes(N, d, M), 16), dtype=torch.uint8, device=dev)
+    pws = torch.empty(max(L.moga_permute_batched_ws_bytes(n, B, M), 16), dtype=torch.uint8, device=dev)
+    aws = torch.empty(L.moga_attn_ws_bytes(N, H, hd), dtype=torch.uint8, device=dev)
+    o = torch.empty((N, H, hd), dtype=torch.float32, device=dev)
+    out = torch.empty((N, H, hd), dtype=torch.bfloat16, device=dev)
+    loss = torch.empty(1, dtype=torch.float64, device=dev)
+    gs, keep = moga.geom_struct(geom)
+    scale = 1.0 / math.sqrt(hd)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        c = moga.check
+        c(L.moga_route(P(x), P(w_r), moga.MOGA_BF16, None, N, d, M, P(g), P(gate), P(rws), rws.numel(), sp), "route")
+        c(L.moga_permute_batched(P(g), n, B, M, P(perm), P(cu), P(counts), P(mx), P(pws), pws.numel(), sp), "permute")
+        c(L.moga_group_attn_batched(P(q), P(k), P(v), n, B, H, hd, P(perm), P(cu), M, P(gate), scale, P(o), None,
+                                    P(aws), aws.numel(), sp), "moga")
+        c(L.stga_attn_batched(P(q), P(k), P(v), B, H, hd, moga.ctypes.byref(gs), scale, P(o), P(aws), aws.numel(), sp),
+          "stga")
+        c(L.visual_attn_mean(P(o), o.numel(), P(out), sp), "mean")
+        c(L.moga_balance_loss_batched(P(counts), B, P(rws), N, M, per.alpha, P(loss), sp), "loss")
+
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    moga.device_status()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(0)
+    torch.cuda.synchronize()
+    sampler.start()
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    moga.device_status()
+    step_ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+    cnt = counts.cpu().numpy()
+    flops = moga_flops(cnt, H, hd) + B * stga_flops(per)
+    pk, pk_kind = peaks()
+    cfg = config_dict(per)
+    cfg.update({"workload": "%s, batch of %d videos, M=20" % (per.name, B), "batch": B, "tokens": N,
+                "sequences_per_gpu": B, "parallelism": "per-video groups in one batch"})
+    line = {
+        "metric": "visual-attn layer fwd tokens/s, batch of videos (bf16)", "value": N / (step_ms * 1e-3),
+        "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic (seeded counter-based generator; no dataset)",
+        "config": cfg, "layer_tflops": flops / (step_ms * 1e-3) / 1e12,
+        "layer_frac_of_peak": flops / (step_ms * 1e-3) / 1e12 / pk["bf16_tflops"],
+        "peak": {"bf16_tflops": pk["bf16_tflops"], "kind": pk_kind}, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    del keep
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -564,11 +652,15 @@ def main():
                     help="run stga_attn_mean (mean inside the STGA frame pass) instead of stga_attn + visual_attn_mean")
     ap.add_argument("--train", action="store_true",
                     help="time the training step (saving forward + backward) instead of the forward")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="time the forward over a batch of this many videos (per-video groups, M=20)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
     if args.train:
         return run_train(args)
+    if args.batch > 0:
+        return run_batch(args)
     return run_ours(args)
 
 
