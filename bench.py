@@ -641,6 +641,90 @@ def run_batch(args):
     return 0
 
 
+def run_sp(args):
+    """Sequence-parallel forward: ONE 5 s Wan-1.3B video sharded over the N ranks
+    (rank r holds tokens [r n, (r+1) n)), routing all-gathered, Q/K/V exchanged
+    to head shards by all-to-all, the layer per head shard, the output
+    exchanged back (sparse_attention_long_moga_b200.sp).  Strong scaling; the
+    step time includes the collectives; max over ranks.  One JSON line."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if not dist.is_initialized():
+        if world == 1:
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", str(29500 + os.getpid() % 1000))
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    import sparse_attention_long_moga_b200 as moga
+    from sparse_attention_long_moga_b200.sp import sp_visual_attention_forward
+    wl = WORKLOAD
+    if wl.H % world or wl.N % world:
+        if rank == 0:
+            print(json.dumps({"metric": "visual-attn layer fwd tokens/s, sequence-parallel (bf16)",
+                              "unavailable": "%d ranks do not divide %d heads and %d tokens" % (world, wl.H, wl.N)}))
+        dist.destroy_process_group()
+        return 0
+    inp = make_inputs(wl)
+    geom = W.stga_shape(wl)
+    n = wl.N // world
+    sl = slice(rank * n, (rank + 1) * n)
+
+    def to_dev(a):
+        t = torch.from_numpy(np.ascontiguousarray(a.view(np.int16) if a.dtype == np.uint16 else a))
+        return t.to(dev).view(torch.bfloat16) if a.dtype == np.uint16 else t.to(dev)
+
+    x, q, k, v = (to_dev(inp[nm][sl]) for nm in ("x", "q", "k", "v"))
+    w_r = to_dev(inp["w_r"])
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        return sp_visual_attention_forward(x, w_r, None, q, k, v, wl.M, geom, wl.alpha)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    moga.device_status()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks = sampler.stop()
+    moga.device_status()
+    local_ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+    step_ms = max_over_ranks(local_ms, device=dev)
+    if rank == 0:
+        cfg = config_dict(wl)
+        cfg.update({"sequences_per_gpu": 1.0 / world, "parallelism": "sequence parallel over %d GPUs (routing "
+                    "all-gather, Q/K/V all-to-all to head shards, output all-to-all back; NCCL)" % world})
+        print(json.dumps({
+            "metric": "visual-attn layer fwd tokens/s, sequence-parallel (bf16)", "value": wl.N / (step_ms * 1e-3),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": True, "scaling": "strong", "dtype": "bf16",
+            "data": "synthetic (seeded counter-based generator; no dataset)", "config": cfg, "clocks": clocks}),
+            flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -652,6 +736,8 @@ def main():
                     help="run stga_attn_mean (mean inside the STGA frame pass) instead of stga_attn + visual_attn_mean")
     ap.add_argument("--train", action="store_true",
                     help="time the training step (saving forward + backward) instead of the forward")
+    ap.add_argument("--sp", action="store_true",
+                    help="sequence-parallel forward of one video over the ranks (strong scaling)")
     ap.add_argument("--batch", type=int, default=0,
                     help="time the forward over a batch of this many videos (per-video groups, M=20)")
     args = ap.parse_args()
@@ -661,6 +747,8 @@ def main():
         return run_train(args)
     if args.batch > 0:
         return run_batch(args)
+    if args.sp:
+        return run_sp(args)
     return run_ours(args)
 
 

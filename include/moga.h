@@ -331,6 +331,34 @@ moga_status stga_attn_batched(const void* q, const void* k, const void* v, int32
 moga_status moga_balance_loss_batched(const int32_t* counts, int32_t B, const void* route_ws, int64_t N,
                                       int32_t M, float alpha, double* loss, void* stream);
 
+/* --------------------------------------------------- sequence parallelism --
+ * P ranks (one GPU each) share one video of N tokens, rank r holding tokens
+ * [r n, (r+1) n), n = N / P (MoGA note, key design 2; translation, 方法:
+ * route the local tokens, which carry every head, collect the routing results
+ * of all tokens, then exchange sequence shards for head shards).  The
+ * collectives belong to the caller; these calls lay out their buffers and
+ * give each rank its share of the loss.  H must be a multiple of P and
+ * (H / P) * hd * 2 a multiple of 16; pointers 16-byte aligned.
+ */
+
+/* src [n][H][hd] bf16 -> dst [P][n][H/P][hd] bf16: chunk j is the slice of
+ * heads [j H/P, (j+1) H/P) of every local token, sent to rank j by an equal-
+ * split all-to-all (which then delivers [N][H/P][hd] in token order). */
+moga_status moga_sp_pack_heads(const void* src, int64_t n, int32_t H, int32_t hd, int32_t P, void* dst,
+                               void* stream);
+
+/* src [P][n][H/P][hd] bf16 (the receive buffer of the return all-to-all:
+ * chunk j holds this rank's n tokens for rank j's heads) -> dst [n][H][hd]. */
+moga_status moga_sp_unpack_heads(const void* src, int64_t n, int32_t H, int32_t hd, int32_t P, void* dst,
+                                 void* stream);
+
+/* This rank's share of L_gb: counts [M] over all N tokens (moga_permute of the
+ * gathered group ids), route_ws from moga_route over the rank's n_local
+ * tokens; F_i and P_i both normalised by N.  The sum over ranks (an
+ * all-reduce) is L_gb.  loss: [1] double, written. */
+moga_status moga_balance_loss_part(const int32_t* counts, const void* route_ws, int64_t n_local, int64_t N,
+                                   int32_t M, float alpha, double* loss, void* stream);
+
 /* ------------------------------------------------------------- diagnostics */
 /* Text of the last host-side error of the calling thread ("" if none). */
 const char* moga_last_error(void);

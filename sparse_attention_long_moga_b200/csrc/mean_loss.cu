@@ -176,3 +176,20 @@ extern "C" moga_status moga_balance_loss_batched(const int32_t* counts, int32_t 
       counts, static_cast<const float*>(route_ws), route_partial_rows(N), (int)N, M, B, alpha, loss);
   return check_launch("moga_balance_loss_batched");
 }
+
+// One rank's share of L_gb under sequence parallelism: F_i from the counts of
+// all N tokens (every rank holds them after the routing all-gather), P_i
+// summed over this rank's n_local tokens only (its router workspace), both
+// normalised by N.  The sum of the ranks' shares is L_gb.
+extern "C" moga_status moga_balance_loss_part(const int32_t* counts, const void* route_ws, int64_t n_local,
+                                              int64_t N, int32_t M, float alpha, double* loss, void* stream) {
+  using namespace moga;
+  if (!counts || !route_ws || !loss) return fail(MOGA_ERR_INVALID_ARG, "moga_balance_loss_part: null pointer");
+  if (N <= 0 || N > INT32_MAX || n_local <= 0 || n_local > N)
+    return fail(MOGA_ERR_INVALID_ARG, "moga_balance_loss_part: n_local=%lld, N=%lld", (long long)n_local,
+                (long long)N);
+  if (M < 1 || M > 32) return fail(MOGA_ERR_INVALID_ARG, "moga_balance_loss_part: M=%d not in [1, 32]", M);
+  mean_detail::balance_loss_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(
+      counts, static_cast<const float*>(route_ws), route_partial_rows(n_local), (int)N, M, 1, alpha, loss);
+  return check_launch("moga_balance_loss_part");
+}

@@ -8,3 +8,4 @@
 #include "attention.cu"
 #include "attention_bwd.cu"
 #include "route_bwd.cu"
+#include "sp.cu"
