@@ -725,6 +725,78 @@ def run_sp(args):
     return 0
 
 
+def run_qkv(args):
+    """The router fused into the Q/K/V projection on the 5 s Wan-1.3B workload (x
+    [32760, 1536] bf16, W_qkv [4608, 1536]): moga_qkv_route timed against the unfused
+    pair it replaces, a library GEMM (torch.matmul, cuBLAS) plus moga_route.  One JSON
+    line (not the headline line)."""
+    import torch
+
+    import sparse_attention_long_moga_b200 as moga
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    wl = WORKLOAD
+    inp = make_inputs(wl)
+    x = torch.from_numpy(inp["x"].view(np.int16)).to(dev).view(torch.bfloat16)
+    w_r = torch.from_numpy(inp["w_r"].view(np.int16)).to(dev).view(torch.bfloat16)
+    wq = np.ascontiguousarray(np.concatenate([W.proj_weight_bits(wl, c) for c in "qkv"], axis=1).T)
+    w_qkv = torch.from_numpy(wq.view(np.int16)).to(dev).view(torch.bfloat16)
+    N, d, H, hd, M = wl.N, wl.d, wl.H, wl.hd, wl.M
+    L = moga._lib.lib()
+    P = moga._ptr
+    sp = moga._stream()
+    q, k, v = (torch.empty((N, H, hd), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    y = torch.empty((N, 3 * H * hd), dtype=torch.bfloat16, device=dev)
+    g = torch.empty(N, dtype=torch.int32, device=dev)
+    gate = torch.empty(N, dtype=torch.float32, device=dev)
+    ws = torch.empty(L.moga_route_ws_bytes(N, d, M), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def fused():
+        moga.check(L.moga_qkv_route(P(x), P(w_qkv), P(w_r), None, N, d, H, hd, M, P(q), P(k), P(v), P(g), P(gate),
+                                    P(ws), ws.numel(), sp), "qkv_route")
+
+    def unfused():
+        torch.matmul(x, w_qkv.t(), out=y)
+        moga.check(L.moga_route(P(x), P(w_r), moga.MOGA_BF16, None, N, d, M, P(g), P(gate), P(ws), ws.numel(), sp),
+                   "route")
+
+    def timeit(fn):
+        for _ in range(args.warmup):
+            flush.zero_()
+            fn()
+        ts = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    sampler = ClockSampler(0)
+    sampler.start()
+    t_f = timeit(fused)
+    t_u = timeit(unfused)
+    clocks = sampler.stop()
+    moga.device_status()
+    flops = 2.0 * N * d * (3 * H * hd + M)
+    pk, pk_kind = peaks()
+    line = {"metric": "Q/K/V projection with the router fused in, tokens/s (bf16)", "value": N / (t_f * 1e-3),
+            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_f,
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic (seeded counter-based generator; no dataset)",
+            "config": {"workload": wl.name + ", x [%d, %d] . W_qkv^T [%d, %d] + router M=%d" % (N, d, 3 * H * hd, d, M)},
+            "fused_tflops": flops / (t_f * 1e-3) / 1e12,
+            "fused_frac_of_peak": flops / (t_f * 1e-3) / 1e12 / pk["bf16_tflops"],
+            "unfused_ms": t_u, "unfused_what": "torch.matmul (cuBLAS) + moga_route",
+            "peak": {"bf16_tflops": pk["bf16_tflops"], "kind": pk_kind}, "clocks": clocks}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -736,6 +808,8 @@ def main():
                     help="run stga_attn_mean (mean inside the STGA frame pass) instead of stga_attn + visual_attn_mean")
     ap.add_argument("--train", action="store_true",
                     help="time the training step (saving forward + backward) instead of the forward")
+    ap.add_argument("--qkv", action="store_true",
+                    help="time the router fused into the Q/K/V projection against GEMM + route")
     ap.add_argument("--sp", action="store_true",
                     help="sequence-parallel forward of one video over the ranks (strong scaling)")
     ap.add_argument("--batch", type=int, default=0,
@@ -749,6 +823,8 @@ def main():
         return run_batch(args)
     if args.sp:
         return run_sp(args)
+    if args.qkv:
+        return run_qkv(args)
     return run_ours(args)
 
 

@@ -331,6 +331,27 @@ moga_status stga_attn_batched(const void* q, const void* k, const void* v, int32
 moga_status moga_balance_loss_batched(const int32_t* counts, int32_t B, const void* route_ws, int64_t N,
                                       int32_t M, float alpha, double* loss, void* stream);
 
+/* ------------------------------------------- router fused into Q/K/V --
+ * The attention layer's Q/K/V projection (the step just before the path)
+ * with the router riding on the same x tiles (MoGA note, key design 1: the
+ * router is a linear projection of the same tokens), so routing needs no
+ * pass of its own over x:
+ *   [q | k | v][t] = W_qkv . x[t]   (fp32 accumulation, bf16 out)
+ *   r = x . W_r (+ bias), p = softmax(r), g = argmax p, gate = p[g]
+ * x:      [N][d] bf16;  w_qkv: [3*H*hd][d] bf16 (a linear layer's weight:
+ *         rows [0, H*hd) for Q, then K, then V);  w_r: [d][M] bf16;
+ *         bias: [M] fp32 or NULL
+ * q, k, v: [N][H][hd] bf16, written;  group_id [N] int32, gate_prob [N]
+ *         fp32, written
+ * ws:     moga_route_ws_bytes(N, d, M) bytes, 256-byte aligned; on return
+ *         it holds the per-32-token sums of p(i|x) that moga_balance_loss
+ *         reads, exactly as after moga_route.
+ * Requires d % 8 == 0, hd in {64, 128}, 1 <= M <= 32, 16-byte aligned x,
+ * w_qkv, q, k, v. */
+moga_status moga_qkv_route(const void* x, const void* w_qkv, const void* w_r, const float* bias, int64_t N,
+                           int32_t d, int32_t H, int32_t hd, int32_t M, void* q, void* k, void* v,
+                           int32_t* group_id, float* gate_prob, void* ws, size_t ws_bytes, void* stream);
+
 /* --------------------------------------------------- sequence parallelism --
  * P ranks (one GPU each) share one video of N tokens, rank r holding tokens
  * [r n, (r+1) n), n = N / P (MoGA note, key design 2; translation, 方法:

@@ -71,6 +71,29 @@ def moga_route(x: torch.Tensor, w_r: torch.Tensor, bias: torch.Tensor | None = N
     return g, gate, ws
 
 
+def moga_qkv_route(x: torch.Tensor, w_qkv: torch.Tensor, w_r: torch.Tensor, bias: torch.Tensor | None, H: int,
+                   hd: int):
+    """The Q/K/V projection with the router fused in: x [N, d] bf16, w_qkv [3*H*hd, d] bf16
+    (a linear layer's weight), w_r [d, M] bf16.  Returns (q, k, v [N, H, hd] bf16, g, gate, ws)."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(w_qkv, torch.bfloat16, "w_qkv", 2)
+    _need(w_r, torch.bfloat16, "w_r", 2)
+    N, d = x.shape
+    M = w_r.shape[1]
+    if w_qkv.shape != (3 * H * hd, d) or w_r.shape[0] != d:
+        raise ValueError("w_qkv must be [3*H*hd, d] and w_r [d, M]")
+    if bias is not None:
+        _need(bias, torch.float32, "bias", 1)
+    L = lib()
+    ws = torch.empty(max(L.moga_route_ws_bytes(N, d, M), 16), dtype=torch.uint8, device=x.device)
+    q, k, v = (torch.empty((N, H, hd), dtype=torch.bfloat16, device=x.device) for _ in range(3))
+    g = torch.empty(N, dtype=torch.int32, device=x.device)
+    gate = torch.empty(N, dtype=torch.float32, device=x.device)
+    check(L.moga_qkv_route(_ptr(x), _ptr(w_qkv), _ptr(w_r), _ptr(bias), N, d, H, hd, M, _ptr(q), _ptr(k), _ptr(v),
+                           _ptr(g), _ptr(gate), _ptr(ws), ws.numel(), _stream()), "moga_qkv_route")
+    return q, k, v, g, gate, ws
+
+
 def moga_permute(group_id: torch.Tensor, M: int):
     """Stable group permute.  Returns (perm [N], cu_seqlens [M+1], counts [M], max_seqlen [1]), int32."""
     _need(group_id, torch.int32, "group_id", 1)

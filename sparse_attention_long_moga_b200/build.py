@@ -14,7 +14,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmoga.so")
 SOURCES = ["moga_lib.cu"]
-DEPS = ["tc_common.cuh", "route_tc.cu", "route_bwd.cu", "sp.cu", "attention_bwd.cu", "api_common.cu", "route.cu", "permute.cu", "permute_noalloc.cu", "mean_loss.cu", "attention.cu", "common.cuh"]
+DEPS = ["tc_common.cuh", "route_tc.cu", "route_bwd.cu", "sp.cu", "qkv_route.cu", "attention_bwd.cu", "api_common.cu", "route.cu", "permute.cu", "permute_noalloc.cu", "mean_loss.cu", "attention.cu", "common.cuh"]
 
 
 def nvcc() -> str:

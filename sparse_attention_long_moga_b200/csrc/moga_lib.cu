@@ -9,3 +9,4 @@
 #include "attention_bwd.cu"
 #include "route_bwd.cu"
 #include "sp.cu"
+#include "qkv_route.cu"

@@ -230,6 +230,14 @@ def qkv_rows_bits(wl: Workload, which: str, rows: np.ndarray, redraw: dict | Non
     return bits if head is not None else bits.reshape(len(rows), wl.H, wl.hd)
 
 
+def proj_weight_bits(wl: Workload, which: str) -> np.ndarray:
+    """bf16 bits of a Q, K or V projection weight [d, H*hd] ~ N(0, 1/d) (the draws of the
+    projected workload's weights, rounded to bf16 as a model's weights would be)."""
+    stream = {"q": S_WQ, "k": S_WK, "v": S_WV}[which]
+    W = rng.normal_block(wl.seed, stream, np.arange(wl.d), wl.H * wl.hd) / math.sqrt(wl.d)
+    return to_bf16_bits(W)
+
+
 def qkv_stored(wl: Workload, which: str, redraw: dict | None = None, chunk: int = 4096) -> np.ndarray:
     out = np.empty((wl.N, wl.H, wl.hd), dtype=np.uint16)
 
