@@ -749,7 +749,7 @@ def run_qkv(args):
     y = torch.empty((N, 3 * H * hd), dtype=torch.bfloat16, device=dev)
     g = torch.empty(N, dtype=torch.int32, device=dev)
     gate = torch.empty(N, dtype=torch.float32, device=dev)
-    ws = torch.empty(L.moga_route_ws_bytes(N, d, M), dtype=torch.uint8, device=dev)
+    ws = torch.empty(L.moga_qkv_route_ws_bytes(N, d, M), dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 

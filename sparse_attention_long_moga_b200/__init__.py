@@ -85,7 +85,7 @@ def moga_qkv_route(x: torch.Tensor, w_qkv: torch.Tensor, w_r: torch.Tensor, bias
     if bias is not None:
         _need(bias, torch.float32, "bias", 1)
     L = lib()
-    ws = torch.empty(max(L.moga_route_ws_bytes(N, d, M), 16), dtype=torch.uint8, device=x.device)
+    ws = torch.empty(max(L.moga_qkv_route_ws_bytes(N, d, M), 16), dtype=torch.uint8, device=x.device)
     q, k, v = (torch.empty((N, H, hd), dtype=torch.bfloat16, device=x.device) for _ in range(3))
     g = torch.empty(N, dtype=torch.int32, device=x.device)
     gate = torch.empty(N, dtype=torch.float32, device=x.device)

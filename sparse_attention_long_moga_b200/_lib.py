@@ -41,6 +41,7 @@ SIGNATURES = {
     "moga_sp_pack_heads": (ctypes.c_int, [_P, _I64, _I32, _I32, _I32, _P, _P]),
     "moga_sp_unpack_heads": (ctypes.c_int, [_P, _I64, _I32, _I32, _I32, _P, _P]),
     "moga_balance_loss_part": (ctypes.c_int, [_P, _P, _I64, _I64, _I32, _F32, _P, _P]),
+    "moga_qkv_route_ws_bytes": (_SZ, [_I64, _I32, _I32]),
     "moga_qkv_route": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ,
                                       _P]),
     "moga_route_train": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _I64, _I32, _I32, _P, _P, _P, _P, _SZ, _P]),

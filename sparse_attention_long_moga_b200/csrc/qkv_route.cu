@@ -6,24 +6,26 @@
 // scores followed by a softmax and an argmax; the Q/K/V projection is the
 // attention layer's own input projection, the step just before the path.
 //
-// Tiles of 128 tokens x 192 output columns; the router's NP (16 or 32)
-// columns ride along with the first column tile of every token tile.  One
-// persistent CTA per SM, 192 threads:
-//   warp 4     producer: TMA of x (128 x 64 k) and W_qkv (192 x 64 k) per
-//              stage, plus W_r^T (NP x 64 k) for router tiles; 4 stages
-//   warp 5     TMEM allocator; lane 0 issues tcgen05.mma: M=128, N=192, K=16
-//              into one of two accumulator buffers (columns 0 and 256), and
-//              for router tiles M=128, N=NP into kSlots slots beside them,
-//              k stage kt going to slot kt % kSlots (each slot sums a few
-//              stages; the epilogue adds the slots in fp32 with round to
-//              nearest, which keeps the logits close to a plain fp32 dot
-//              product: the tensor core's accumulation does not round to
-//              nearest)
-//   warps 0-3  epilogue, thread = token row = TMEM lane: 192 accumulator
-//              columns -> bf16 -> the token's q, k or v row (16-byte stores),
-//              then for router tiles the router epilogue (bias, softmax,
-//              argmax with the lowest index on a tie, gate, per-32-token
-//              sums of p(i|x) for L_gb, in the layout moga_route writes)
+// Tiles of 128 tokens x 256 columns of the product.  The first column tile of
+// every token tile holds output columns [0, 192) and the router's 64 columns;
+// the others hold 256 output columns each.  The router's columns form S slots
+// of NP (S = 64 / NP): its weight is expanded once (a small kernel) into a
+// [64][d] matrix whose slot-s rows carry W_r^T only on the k stages with
+// (k / 64) % S == s and zeros elsewhere, so the one N = 256 product per k step
+// adds every stage into its own slot (adding the zero rows is exact).  The
+// epilogue adds the S slots in fp32 with round to nearest: the tensor core's
+// fp32 accumulation does not round to nearest, and splitting the sum keeps
+// the logits close to a plain fp32 dot product.  One persistent CTA per SM,
+// 192 threads:
+//   warp 4     producer: TMA of x (128 x 64 k) and of the tile's 256 B rows
+//              (W_qkv rows, plus the expanded router rows for first tiles)
+//   warp 5     TMEM allocator; lane 0 issues tcgen05.mma (M=128, N=256,
+//              K=16) into one of two accumulator buffers (columns 0, 256)
+//   warps 0-3  epilogue, thread = token row = TMEM lane: accumulator columns
+//              -> bf16 -> the token's q, k or v row (16-byte stores), and for
+//              first tiles the router epilogue (bias, softmax, argmax with
+//              the lowest index on a tie, gate, per-32-token sums of p(i|x)
+//              for L_gb, in the layout moga_route writes)
 // The two accumulator buffers let the epilogue of one tile overlap the
 // products of the next.  All waits are bounded.
 namespace moga {
@@ -31,39 +33,43 @@ namespace qkv {
 
 using namespace moga::tc;
 
-constexpr int BM = 128, BN = 192, BK = 64;
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int kRouterCols = 64;          // router columns of a first tile
+constexpr int kFirstCols = BN - kRouterCols;   // 192 output columns in a first tile
 constexpr int kStages = 4;
 constexpr int kThreads = 192;
-constexpr int kXBytes = BM * 128;      // 16 KB
-constexpr int kWBytes = BN * 128;      // 24 KB
-// TMEM: accumulator buffers at columns 0 and 256 (192 columns each); the
-// router slots fill the two 64-column gaps [192, 256) and [448, 512)
-constexpr int kAccStride = 256;
-constexpr int kRouterCols = 2 * (kAccStride - BN);   // 128 columns of router slots
+constexpr int kXBytes = BM * 128;        // 16 KB
+constexpr int kBBytes = BN * 128;        // 32 KB
+constexpr int kStageBytes = kXBytes + kBBytes;
+constexpr int kBarOff = kStages * kStageBytes;
+constexpr int kMiscOff = kBarOff + 32 * 8;
+constexpr int kSmemBytes = kMiscOff + 64 + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
-template <int NP>
-struct Cfg {
-  static constexpr int kSlots = kRouterCols / NP;          // 8 or 4
-  static constexpr int kHalf = kSlots / 2;                 // slots per gap
-  __device__ static uint32_t slot_col(int s) {
-    return (uint32_t)((s < kHalf ? BN : kAccStride + BN) + (s % kHalf) * NP);
+// first output column of column tile n (tile 0 is a first tile)
+__host__ __device__ inline int tile_col0(int n) { return n == 0 ? 0 : kFirstCols + (n - 1) * BN; }
+
+// wx[s * NP + m][k] = W_r[k][m] if m < M, k < d and (k / 64) % S == s, else 0;
+// [64][dpad] bf16 (S = 64 / NP slots of NP columns)
+__global__ void __launch_bounds__(256)
+prep_router_kernel(const __nv_bfloat16* __restrict__ w_r, int d, int M, int NP, int dpad,
+                   __nv_bfloat16* __restrict__ wx) {
+  const int S = kRouterCols / NP;
+  const int total = kRouterCols * dpad;
+  for (int i = blockIdx.x * 256 + threadIdx.x; i < total; i += gridDim.x * 256) {
+    const int row = i / dpad, k = i - row * dpad;
+    const int s = row / NP, m = row - s * NP;
+    const bool on = m < M && k < d && (k / BK) % S == s;
+    wx[i] = on ? w_r[(size_t)k * M + m] : __float2bfloat16(0.f);
   }
-  static constexpr int kRBytes = NP * 128;
-  static constexpr int kStageBytes = kXBytes + kWBytes + kRBytes;   // multiple of 1024
-  static constexpr int kBarOff = kStages * kStageBytes;
-  static constexpr int kMiscOff = kBarOff + 32 * 8;
-  static constexpr int kSmemBytes = kMiscOff + 64 + 1024;
-  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
-};
+}
 
 // barriers
 constexpr int Q_FULL = 0;                 // [kStages]
 constexpr int Q_EMPTY = kStages;          // [kStages]
 constexpr int Q_ACC_FULL = 2 * kStages;   // [2]
 constexpr int Q_ACC_EMPTY = Q_ACC_FULL + 2;   // [2] (128 arrivals)
-constexpr int Q_R_FULL = Q_ACC_EMPTY + 2;
-constexpr int Q_R_EMPTY = Q_R_FULL + 1;   // 128 arrivals
-constexpr int Q_END = Q_R_EMPTY + 1;
+constexpr int Q_END = Q_ACC_EMPTY + 2;
 static_assert(Q_END < 32, "barrier area");
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -82,16 +88,37 @@ struct Params {
   long long timeout;
 };
 
+// bf16 of 32 accumulator columns [c0, c0 + 32) of the tile into the token's
+// q / k / v row (output columns past n_out skipped; 8 columns never straddle
+// q, k and v since H * hd is a multiple of 64)
+__device__ __forceinline__ void store_cols(const Params& p, int tok, int col0, const float* v) {
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int col = col0 + 8 * e;
+    if (col < p.n_out) {
+      const int which = col / p.hhd, rem = col - which * p.hhd;
+      __nv_bfloat16* dst = (which == 0 ? p.q : which == 1 ? p.k : p.v) + (size_t)tok * p.hhd + rem;
+      uint4 pk;
+      pk.x = pack_bf16x2(v[8 * e], v[8 * e + 1]);
+      pk.y = pack_bf16x2(v[8 * e + 2], v[8 * e + 3]);
+      pk.z = pack_bf16x2(v[8 * e + 4], v[8 * e + 5]);
+      pk.w = pack_bf16x2(v[8 * e + 6], v[8 * e + 7]);
+      *reinterpret_cast<uint4*>(dst) = pk;
+    }
+  }
+}
+
 template <int NP>
 __global__ void __launch_bounds__(kThreads, 1)
 qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tm_x,
-                 const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_r) {
-  using C = Cfg<NP>;
+                 const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w,
+                 const __grid_constant__ CUtensorMap tm_r) {
+  constexpr int S = kRouterCols / NP;     // router slots
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  auto bar = [&](int i) { return sbase + C::kBarOff + 8u * (uint32_t)i; };
-  int* misc = reinterpret_cast<int*>(smem + C::kMiscOff);
+  auto bar = [&](int i) { return sbase + kBarOff + 8u * (uint32_t)i; };
+  int* misc = reinterpret_cast<int*>(smem + kMiscOff);
   volatile int* abort_flag = misc;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -108,8 +135,6 @@ qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
       mbar_init(bar(Q_ACC_FULL + b), 1);
       mbar_init(bar(Q_ACC_EMPTY + b), BM);
     }
-    mbar_init(bar(Q_R_FULL), 1);
-    mbar_init(bar(Q_R_EMPTY), BM);
     mbar_init(bar(Q_END), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -128,6 +153,7 @@ qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_x)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_w0)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_w)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_r)) : "memory");
       int c = 0;
@@ -136,15 +162,18 @@ qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles_total && ok; t += gridDim.x) {
         const int m = t / p.n_tiles, n = t - m * p.n_tiles;
-        const bool router = n == 0;
         for (int kt = 0; kt < p.n_k; ++kt, ++c) {
           const int st = c % kStages;
           if (!(ok = mbar_wait(bar(Q_EMPTY + st), ((c / kStages) & 1) ^ 1, abort_flag, timeout))) break;
-          mbar_arrive_expect_tx(bar(Q_FULL + st), kXBytes + kWBytes + (router ? C::kRBytes : 0));
-          const uint32_t dst = sbase + st * C::kStageBytes;
+          mbar_arrive_expect_tx(bar(Q_FULL + st), kStageBytes);
+          const uint32_t dst = sbase + st * kStageBytes;
           tma_load_2d(dst, &tm_x, kt * BK, m * BM, bar(Q_FULL + st));
-          tma_load_2d(dst + kXBytes, &tm_w, kt * BK, n * BN, bar(Q_FULL + st));
-          if (router) tma_load_2d(dst + kXBytes + kWBytes, &tm_r, kt * BK, 0, bar(Q_FULL + st));
+          if (n == 0) {
+            tma_load_2d(dst + kXBytes, &tm_w0, kt * BK, 0, bar(Q_FULL + st));
+            tma_load_2d(dst + kXBytes + kFirstCols * 128, &tm_r, kt * BK, 0, bar(Q_FULL + st));
+          } else {
+            tma_load_2d(dst + kXBytes, &tm_w, kt * BK, tile_col0(n), bar(Q_FULL + st));
+          }
           last[st] = c;
         }
       }
@@ -155,41 +184,26 @@ qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
   } else if (warp == 5) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_w = instr_desc(BN, false);
-      constexpr uint32_t idesc_r = instr_desc(NP, false);
-      int c = 0, j = 0, nr = 0;   // stage, local tile and router tile counters
+      constexpr uint32_t idesc = instr_desc(BN, false);
+      int c = 0, j = 0;   // stage and local tile counters
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles_total && ok; t += gridDim.x, ++j) {
-        const int n = t % p.n_tiles;
-        const bool router = n == 0;
         const int b = j & 1;
         if (!(ok = mbar_wait(bar(Q_ACC_EMPTY + b), ((j >> 1) & 1) ^ 1, abort_flag, timeout))) break;
-        if (router && !(ok = mbar_wait(bar(Q_R_EMPTY), (nr & 1) ^ 1, abort_flag, timeout))) break;
-        const uint32_t acc = tmem + b * kAccStride;
+        const uint32_t acc = tmem + b * BN;
         for (int kt = 0; kt < p.n_k; ++kt, ++c) {
           const int st = c % kStages;
           if (!(ok = mbar_wait(bar(Q_FULL + st), (c / kStages) & 1, abort_flag, timeout))) break;
           tc_fence_after();
-          const uint32_t xa = sbase + st * C::kStageBytes, wa = xa + kXBytes, ra = wa + kWBytes;
+          const uint32_t xa = sbase + st * kStageBytes, ba = xa + kXBytes;
 #pragma unroll
           for (int ks = 0; ks < BK / 16; ++ks)
-            tc_mma_ss(acc, smem_desc(xa + ks * 32, 16, 1024), smem_desc(wa + ks * 32, 16, 1024), idesc_w,
+            tc_mma_ss(acc, smem_desc(xa + ks * 32, 16, 1024), smem_desc(ba + ks * 32, 16, 1024), idesc,
                       (kt > 0 || ks > 0) ? 1u : 0u);
-          if (router) {
-            const uint32_t slot = tmem + C::slot_col(kt % C::kSlots);
-#pragma unroll
-            for (int ks = 0; ks < BK / 16; ++ks)
-              tc_mma_ss(slot, smem_desc(xa + ks * 32, 16, 1024), smem_desc(ra + ks * 32, 16, 1024), idesc_r,
-                        (kt >= C::kSlots || ks > 0) ? 1u : 0u);
-          }
           tc_commit(bar(Q_EMPTY + st));
         }
         if (!ok) break;
         tc_commit(bar(Q_ACC_FULL + b));
-        if (router) {
-          tc_commit(bar(Q_R_FULL));
-          ++nr;
-        }
       }
       tc_commit(bar(Q_END));
       mbar_drain(bar(Q_END), 0, timeout);
@@ -202,8 +216,7 @@ qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
     float bias[NP];
 #pragma unroll
     for (int mm = 0; mm < NP; ++mm) bias[mm] = (p.bias && mm < p.M) ? __ldg(p.bias + mm) : 0.f;
-    const int used_slots = min(C::kSlots, p.n_k);
-    int j = 0, nr = 0;
+    int j = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < n_tiles_total && ok; t += gridDim.x, ++j) {
       const int m = t / p.n_tiles, n = t - m * p.n_tiles;
@@ -212,48 +225,34 @@ qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
       tc_fence_after();
       const int tok = m * BM + row;
       const bool in = tok < p.N;
+      const uint32_t acc = tmem + lane_addr + b * BN;
+      const int ncols = n == 0 ? kFirstCols : BN;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int c0 = 0; c0 < ncols; c0 += 32) {
         float v[32];
-        tmem_ld32(tmem + lane_addr + b * kAccStride + c0, v);
+        tmem_ld32(acc + c0, v);
         tmem_wait_ld();
-        if (in) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int col = n * BN + c0 + 8 * e;   // 8 columns = 16 bytes, never across q|k|v
-            if (col < p.n_out) {
-              const int which = col / p.hhd, rem = col - which * p.hhd;
-              __nv_bfloat16* dst = (which == 0 ? p.q : which == 1 ? p.k : p.v) + (size_t)tok * p.hhd + rem;
-              uint4 pk;
-              pk.x = pack_bf16x2(v[8 * e], v[8 * e + 1]);
-              pk.y = pack_bf16x2(v[8 * e + 2], v[8 * e + 3]);
-              pk.z = pack_bf16x2(v[8 * e + 4], v[8 * e + 5]);
-              pk.w = pack_bf16x2(v[8 * e + 6], v[8 * e + 7]);
-              *reinterpret_cast<uint4*>(dst) = pk;
-            }
-          }
-        }
+        if (in) store_cols(p, tok, tile_col0(n) + c0, v);
       }
+      if (n != 0) {
+        tc_fence_before();
+        mbar_arrive(bar(Q_ACC_EMPTY + b));
+        continue;
+      }
+      // router: S slots of NP logits in columns [192, 256), added in order
+      float rs[kRouterCols];
+      tmem_ld32(acc + kFirstCols, rs);
+      tmem_ld32(acc + kFirstCols + 32, rs + 32);
+      tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(Q_ACC_EMPTY + b));
-      if (n != 0) continue;
-      // router epilogue for the tile's 128 tokens
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_R_FULL), nr & 1, abort_flag, timeout)))) break;
-      ++nr;
-      tc_fence_after();
       float r[NP];
 #pragma unroll
-      for (int mm = 0; mm < NP; ++mm) r[mm] = 0.f;
-      for (int s = 0; s < used_slots; ++s) {
-        float sv[NP];
-        if constexpr (NP == 16) tmem_ld16(tmem + lane_addr + C::slot_col(s), sv);
-        else tmem_ld32(tmem + lane_addr + C::slot_col(s), sv);
-        tmem_wait_ld();
+      for (int mm = 0; mm < NP; ++mm) {
+        r[mm] = rs[mm];
 #pragma unroll
-        for (int mm = 0; mm < NP; ++mm) r[mm] += sv[mm];
+        for (int s = 1; s < S; ++s) r[mm] += rs[s * NP + mm];
       }
-      tc_fence_before();
-      mbar_arrive(bar(Q_R_EMPTY));
       float pr[NP];
       if (in) {
         float best = -INFINITY;
@@ -288,10 +287,10 @@ qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
 #pragma unroll
         for (int mm = 0; mm < NP; ++mm) {
           if (mm < p.M) {
-            float s = pr[mm];
+            float sum = pr[mm];
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-            if (lane == 0) dst[mm] = s;
+            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+            if (lane == 0) dst[mm] = sum;
           }
         }
       }
@@ -304,25 +303,31 @@ qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
   if (warp == 5) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512u) : "memory");
 }
 
+inline size_t router_bytes(int d) { return (size_t)kRouterCols * route_tc::dpad_of(d) * 2; }
+
 template <int NP>
-static moga_status launch_np(const Params& prm, const void* x, const void* w_qkv, const void* wt, int dpad,
+static moga_status launch_np(const Params& prm, const void* x, const void* w_qkv, const void* wx, int dpad,
                              cudaStream_t s) {
-  using C = Cfg<NP>;
-  CUtensorMap mx, mw, mr;
+  CUtensorMap mx, mw0, mw, mr;
   moga_status st;
   if ((st = route_tc::make_map(&mx, x, prm.N, prm.d, (int64_t)prm.d * 2, BM)) != MOGA_OK) return st;
+  if ((st = route_tc::make_map(&mw0, w_qkv, prm.n_out, prm.d, (int64_t)prm.d * 2, kFirstCols)) != MOGA_OK) return st;
   if ((st = route_tc::make_map(&mw, w_qkv, prm.n_out, prm.d, (int64_t)prm.d * 2, BN)) != MOGA_OK) return st;
-  if ((st = route_tc::make_map(&mr, wt, NP, dpad, (int64_t)dpad * 2, NP)) != MOGA_OK) return st;
-  cudaError_t e = cudaFuncSetAttribute(qkv_route_kernel<NP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::kSmemBytes);
+  if ((st = route_tc::make_map(&mr, wx, kRouterCols, dpad, (int64_t)dpad * 2, kRouterCols)) != MOGA_OK) return st;
+  cudaError_t e = cudaFuncSetAttribute(qkv_route_kernel<NP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return fail(MOGA_ERR_CUDA, "moga_qkv_route: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
   const int grid = std::min(prm.m_tiles * prm.n_tiles, route_tc::sm_count());
-  qkv_route_kernel<NP><<<grid, kThreads, C::kSmemBytes, s>>>(prm, mx, mw, mr);
+  qkv_route_kernel<NP><<<grid, kThreads, kSmemBytes, s>>>(prm, mx, mw0, mw, mr);
   return check_launch("moga_qkv_route");
 }
 
 }  // namespace qkv
 }  // namespace moga
+
+extern "C" size_t moga_qkv_route_ws_bytes(int64_t N, int32_t d, int32_t M) {
+  if (N <= 0 || N > INT32_MAX || M < 1 || M > 32 || d <= 0 || d % 8 != 0) return 0;
+  return moga::route_partial_bytes(N, M) + moga::qkv::router_bytes(d);
+}
 
 extern "C" moga_status moga_qkv_route(const void* x, const void* w_qkv, const void* w_r, const float* bias,
                                       int64_t N, int32_t d, int32_t H, int32_t hd, int32_t M, void* q, void* k,
@@ -342,15 +347,16 @@ extern "C" moga_status moga_qkv_route(const void* x, const void* w_qkv, const vo
                       reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
                       reinterpret_cast<uintptr_t>(v);
   if (a & 15) return fail(MOGA_ERR_INVALID_ARG, "moga_qkv_route: x, w_qkv, q, k, v must be 16-byte aligned");
-  const size_t need = moga_route_ws_bytes(N, d, M);
+  const size_t need = moga_qkv_route_ws_bytes(N, d, M);
   if (ws_bytes < need) return fail(MOGA_ERR_WORKSPACE, "moga_qkv_route: workspace %zu < %zu bytes", ws_bytes, need);
   if (reinterpret_cast<uintptr_t>(ws) & 255)
     return fail(MOGA_ERR_INVALID_ARG, "moga_qkv_route: workspace not 256-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int dpad = route_tc::dpad_of(d);
-  void* wt = static_cast<uint8_t*>(ws) + route_partial_bytes(N, M);
-  route_tc::prep_wt_kernel<<<ceil_div(route_tc::NPMAX * dpad, 256), 256, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(w_r), d, M, dpad, static_cast<__nv_bfloat16*>(wt));
+  const int NP = M <= 16 ? 16 : 32;
+  void* wx = static_cast<uint8_t*>(ws) + route_partial_bytes(N, M);
+  qkv::prep_router_kernel<<<ceil_div(qkv::kRouterCols * dpad, 256), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(w_r), d, M, NP, dpad, static_cast<__nv_bfloat16*>(wx));
   moga_status st = check_launch("moga_qkv_route/prep");
   if (st != MOGA_OK) return st;
   qkv::Params prm;
@@ -361,7 +367,7 @@ extern "C" moga_status moga_qkv_route(const void* x, const void* w_qkv, const vo
   prm.n_out = 3 * H * hd;
   prm.n_k = dpad / qkv::BK;
   prm.m_tiles = ceil_div((int)N, qkv::BM);
-  prm.n_tiles = ceil_div(prm.n_out, qkv::BN);
+  prm.n_tiles = 1 + ceil_div(prm.n_out - qkv::kFirstCols, qkv::BN);
   prm.bias = bias;
   prm.q = static_cast<__nv_bfloat16*>(q);
   prm.k = static_cast<__nv_bfloat16*>(k);
@@ -370,5 +376,5 @@ extern "C" moga_status moga_qkv_route(const void* x, const void* w_qkv, const vo
   prm.gate_prob = gate_prob;
   prm.partial = static_cast<float*>(ws);
   prm.timeout = 4000000000LL;
-  return M <= 16 ? qkv::launch_np<16>(prm, x, w_qkv, wt, dpad, s) : qkv::launch_np<32>(prm, x, w_qkv, wt, dpad, s);
+  return NP == 16 ? qkv::launch_np<16>(prm, x, w_qkv, wx, dpad, s) : qkv::launch_np<32>(prm, x, w_qkv, wx, dpad, s);
 }
