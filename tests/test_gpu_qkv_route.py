@@ -1,11 +1,12 @@
 """GPU parity of the router fused into the Q/K/V projection against the oracle.
 
-Q, K, V: the kernel accumulates in fp32 and rounds to bf16; the oracle's
-fp64 product rounded to bf16 must agree on all but the elements that sit
-within the fp32 accumulation error of a rounding boundary (at most 1e-3 of
-them), and every element must lie within one bf16 rounding of the fp64
-value plus the fp32 accumulation bound 2^-20 * sum_k |x_k w_k| (which
-covers results that cancel to near zero).  Routing: group ids
+Q, K, V: the kernel accumulates in fp32 (the tensor core's accumulation
+truncates: up to one unit in the last place per K = 16 step) and rounds to
+bf16.  Every element must lie within one bf16 unit of the fp64 product plus
+the accumulation bound (d / 16) * 2^-23 * sum_k |x_k w_k| (which also covers
+results that cancel to near zero); the elements whose bf16 value differs from
+the rounded fp64 product are those near a rounding boundary, a share that
+grows with d (2.8e-3 at d = 5120), checked to stay below 1e-2.  Routing: group ids
 bit-exact (inputs pass the 1e-3 router-margin filter), the gate within 1e-5
 relative, and the per-32-token sums it leaves in the workspace give the
 balance loss within 1e-5 of the oracle's.
@@ -27,6 +28,9 @@ CASES = {
                                       win_h=8, win_w=25, seed=11),
     "tiny_bf16_m20": W.Workload("qkv_tiny_m20", T=8, h=16, w=16, d=128, H=2, hd=128, M=20, shots=(8,), tg_max=0,
                                 win_h=8, win_w=8, seed=12),
+    # the widest router input of the suite: 80 k stages, 20 per router slot
+    "d5120_m5": W.Workload("qkv_d5120", T=4, h=16, w=16, d=5120, H=2, hd=128, M=5, shots=(4,), tg_max=0, win_h=8,
+                           win_w=8, seed=13),
     "wan1.3b_32k": W.WAN13B_5S,
 }
 
@@ -56,9 +60,9 @@ def test_qkv_route_matches_oracle(name, cuda_device):
     for got, ref, mag, which in ((q, rq, mags[0], "q"), (k, rk, mags[1], "k"), (v, rv, mags[2], "v")):
         gb = got.view(torch.int16).cpu().numpy().view(np.uint16)
         diff = gb != W.to_bf16_bits(ref)
-        assert diff.mean() <= 1e-3, "%s %s: %.2e of the elements differ" % (name, which, diff.mean())
+        assert diff.mean() <= 1e-2, "%s %s: %.2e of the elements differ" % (name, which, diff.mean())
         err = np.abs(W.bf16_bits_to_f64(gb) - ref)
-        bound = 2.0 ** -8 * np.abs(ref) + 2.0 ** -20 * mag
+        bound = 2.0 ** -8 * np.abs(ref) + (wl.d / 16) * 2.0 ** -23 * mag
         assert np.all(err <= bound), "%s %s: worst error / bound %.3f" % (name, which, float(np.max(err / bound)))
     rg, rpg, rp = case.route64()
     assert np.array_equal(g.cpu().numpy(), rg)
