@@ -6,40 +6,45 @@
 // scores followed by a softmax and an argmax; the Q/K/V projection is the
 // attention layer's own input projection, the step just before the path.
 //
-// Tiles of 128 tokens x 256 columns of the product.  The first column tile of
-// every token tile holds output columns [0, 192) and the router's 64 columns;
-// the others hold 256 output columns each.  The router's columns form S slots
-// of NP (S = 64 / NP): its weight is expanded once (a small kernel) into a
-// [64][d] matrix whose slot-s rows carry W_r^T only on the k stages with
-// (k / 64) % S == s and zeros elsewhere, so the one N = 256 product per k step
-// adds every stage into its own slot (adding the zero rows is exact).  The
-// epilogue adds the S slots in fp32 with round to nearest: the tensor core's
-// fp32 accumulation does not round to nearest, and splitting the sum keeps
-// the logits close to a plain fp32 dot product.  One persistent CTA per SM,
-// 192 threads:
-//   warp 4     producer: TMA of x (128 x 64 k) and of the tile's 256 B rows
-//              (W_qkv rows, plus the expanded router rows for first tiles)
-//   warp 5     TMEM allocator; lane 0 issues tcgen05.mma (M=128, N=256,
-//              K=16) into one of two accumulator buffers (columns 0, 256)
+// The product runs on pairs of SMs (a cluster of two CTAs, tcgen05
+// cta_group::2): one tile is 256 tokens x 256 columns, each CTA of the pair
+// holding 128 of the tokens (its x rows) and 128 of the 256 B rows, so each
+// SM streams half of the B tile through its shared memory; the leader CTA
+// issues M = 256 products and each CTA's TMEM receives its 128 rows.  The
+// first column tile of every token tile holds output columns [0, 192) and the
+// router's 64 columns; the others hold 256 output columns each.  The
+// router's columns form S slots of NP (S = 64 / NP): its weight is expanded
+// once (a small kernel) into a [64][d] matrix whose slot-s rows carry W_r^T
+// only on the k stages with (k / 64) % S == s and zeros elsewhere, so the
+// product adds every stage into its own slot (adding the zero rows is exact).
+// The epilogue adds the S slots in fp32 with round to nearest: the tensor
+// core's fp32 accumulation does not round to nearest, and splitting the sum
+// keeps the logits close to a plain fp32 dot product.  192 threads per CTA:
+//   warp 4     producer: TMA of this CTA's x rows (128 x 64 k) and B rows
+//              (128 x 64 k), completing on the leader's stage barrier
+//   warp 5     TMEM allocator (both CTAs); in the leader, lane 0 issues
+//              tcgen05.mma.cta_group::2 (M=256, N=256, K=16) into one of two
+//              accumulator buffers (columns 0, 256) and commits to both CTAs
 //   warps 0-3  epilogue, thread = token row = TMEM lane: accumulator columns
 //              -> bf16 -> the token's q, k or v row (16-byte stores), and for
 //              first tiles the router epilogue (bias, softmax, argmax with
 //              the lowest index on a tie, gate, per-32-token sums of p(i|x)
-//              for L_gb, in the layout moga_route writes)
+//              for L_gb, in the layout moga_route writes); then they release
+//              the buffer on the leader's barrier
 // The two accumulator buffers let the epilogue of one tile overlap the
-// products of the next.  All waits are bounded.
+// products of the next.  All mbarrier waits are bounded.
 namespace moga {
 namespace qkv {
 
 using namespace moga::tc;
 
-constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int BM = 128, BN = 256, BK = 64;   // BM: token rows per CTA (256 per pair)
 constexpr int kRouterCols = 64;          // router columns of a first tile
 constexpr int kFirstCols = BN - kRouterCols;   // 192 output columns in a first tile
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr int kThreads = 192;
 constexpr int kXBytes = BM * 128;        // 16 KB
-constexpr int kBBytes = BN * 128;        // 32 KB
+constexpr int kBBytes = (BN / 2) * 128;  // 16 KB: this CTA's half of the B rows
 constexpr int kStageBytes = kXBytes + kBBytes;
 constexpr int kBarOff = kStages * kStageBytes;
 constexpr int kMiscOff = kBarOff + 32 * 8;
@@ -108,10 +113,57 @@ __device__ __forceinline__ void store_cols(const Params& p, int tok, int col0, c
   }
 }
 
+// ---- SM-pair (cta_group::2) primitives
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// address of the same shared-memory object in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// arrive on an mbarrier of any CTA of the cluster (cluster-window address)
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+// tiled 2-D TMA load into this CTA's shared memory, completing on an mbarrier
+// of either CTA of the pair (cluster-window address); no multicast
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0;"
+      " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// arrive once on the barrier at this offset in both CTAs when the leader's
+// earlier products have completed
+__device__ __forceinline__ void commit_pair(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"((uint16_t)3)
+      : "memory");
+}
+constexpr uint32_t kIdescPair = (instr_desc(BN, false) & ~(0x1Fu << 24)) | ((uint32_t)(2 * BM >> 4) << 24);
+
 template <int NP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tm_x,
-                 const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w,
+                 const __grid_constant__ CUtensorMap tm_w128, const __grid_constant__ CUtensorMap tm_w64,
                  const __grid_constant__ CUtensorMap tm_r) {
   constexpr int S = kRouterCols / NP;     // router slots
   extern __shared__ uint8_t smem_raw[];
@@ -123,7 +175,10 @@ qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long timeout = p.timeout;
-  const int n_tiles_total = p.m_tiles * p.n_tiles;
+  const uint32_t rank = cluster_rank();          // 0: leader, 1: peer
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const int n_tiles_total = p.m_tiles * p.n_tiles;   // m_tiles counts 256-token tiles
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -133,19 +188,20 @@ qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(Q_ACC_FULL + b), 1);
-      mbar_init(bar(Q_ACC_EMPTY + b), BM);
+      mbar_init(bar(Q_ACC_EMPTY + b), 2 * BM);
     }
     mbar_init(bar(Q_END), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 5) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(512u)
                  : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();   // both CTAs' barriers are initialised before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -153,41 +209,40 @@ qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_x)) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_w0)) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_w)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_w128)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_w64)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_r)) : "memory");
       int c = 0;
-      int last[kStages];
-      for (int s = 0; s < kStages; ++s) last[s] = -1;
       bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles_total && ok; t += gridDim.x) {
+      for (int t = pair; t < n_tiles_total && ok; t += n_pairs) {
         const int m = t / p.n_tiles, n = t - m * p.n_tiles;
+        const int xrow = m * 2 * BM + (int)rank * BM;
         for (int kt = 0; kt < p.n_k; ++kt, ++c) {
           const int st = c % kStages;
           if (!(ok = mbar_wait(bar(Q_EMPTY + st), ((c / kStages) & 1) ^ 1, abort_flag, timeout))) break;
-          mbar_arrive_expect_tx(bar(Q_FULL + st), kStageBytes);
+          const uint32_t full_leader = peer_addr(bar(Q_FULL + st), 0);
+          // the leader's barrier expects both CTAs' bytes
+          if (leader) mbar_arrive_expect_tx(bar(Q_FULL + st), 2 * kStageBytes);
           const uint32_t dst = sbase + st * kStageBytes;
-          tma_load_2d(dst, &tm_x, kt * BK, m * BM, bar(Q_FULL + st));
-          if (n == 0) {
-            tma_load_2d(dst + kXBytes, &tm_w0, kt * BK, 0, bar(Q_FULL + st));
-            tma_load_2d(dst + kXBytes + kFirstCols * 128, &tm_r, kt * BK, 0, bar(Q_FULL + st));
-          } else {
-            tma_load_2d(dst + kXBytes, &tm_w, kt * BK, tile_col0(n), bar(Q_FULL + st));
+          tma_load_2d_pair(dst, &tm_x, kt * BK, xrow, full_leader);
+          if (n != 0) {
+            tma_load_2d_pair(dst + kXBytes, &tm_w128, kt * BK, tile_col0(n) + (int)rank * (BN / 2), full_leader);
+          } else if (leader) {   // W rows [0, 128)
+            tma_load_2d_pair(dst + kXBytes, &tm_w128, kt * BK, 0, full_leader);
+          } else {               // W rows [128, 192) and the 64 router rows
+            tma_load_2d_pair(dst + kXBytes, &tm_w64, kt * BK, BN / 2, full_leader);
+            tma_load_2d_pair(dst + kXBytes + 64 * 128, &tm_r, kt * BK, 0, full_leader);
           }
-          last[st] = c;
         }
       }
-      for (int s = 0; s < kStages; ++s)
-        if (last[s] >= 0) mbar_drain(bar(Q_FULL + s), (last[s] / kStages) & 1, timeout);
     }
     __syncwarp();
   } else if (warp == 5) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = instr_desc(BN, false);
+    // ------------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
       int c = 0, j = 0;   // stage and local tile counters
       bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles_total && ok; t += gridDim.x, ++j) {
+      for (int t = pair; t < n_tiles_total && ok; t += n_pairs, ++j) {
         const int b = j & 1;
         if (!(ok = mbar_wait(bar(Q_ACC_EMPTY + b), ((j >> 1) & 1) ^ 1, abort_flag, timeout))) break;
         const uint32_t acc = tmem + b * BN;
@@ -198,14 +253,14 @@ qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
           const uint32_t xa = sbase + st * kStageBytes, ba = xa + kXBytes;
 #pragma unroll
           for (int ks = 0; ks < BK / 16; ++ks)
-            tc_mma_ss(acc, smem_desc(xa + ks * 32, 16, 1024), smem_desc(ba + ks * 32, 16, 1024), idesc,
-                      (kt > 0 || ks > 0) ? 1u : 0u);
-          tc_commit(bar(Q_EMPTY + st));
+            mma_pair(acc, smem_desc(xa + ks * 32, 16, 1024), smem_desc(ba + ks * 32, 16, 1024), kIdescPair,
+                     (kt > 0 || ks > 0) ? 1u : 0u);
+          commit_pair(bar(Q_EMPTY + st));
         }
         if (!ok) break;
-        tc_commit(bar(Q_ACC_FULL + b));
+        commit_pair(bar(Q_ACC_FULL + b));
       }
-      tc_commit(bar(Q_END));
+      commit_pair(bar(Q_END));
       mbar_drain(bar(Q_END), 0, timeout);
     }
     __syncwarp();
@@ -218,14 +273,15 @@ qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
     for (int mm = 0; mm < NP; ++mm) bias[mm] = (p.bias && mm < p.M) ? __ldg(p.bias + mm) : 0.f;
     int j = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < n_tiles_total && ok; t += gridDim.x, ++j) {
+    for (int t = pair; t < n_tiles_total && ok; t += n_pairs, ++j) {
       const int m = t / p.n_tiles, n = t - m * p.n_tiles;
       const int b = j & 1;
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_ACC_FULL + b), (j >> 1) & 1, abort_flag, timeout)))) break;
       tc_fence_after();
-      const int tok = m * BM + row;
+      const int tok = m * 2 * BM + (int)rank * BM + row;
       const bool in = tok < p.N;
       const uint32_t acc = tmem + lane_addr + b * BN;
+      const uint32_t empty_leader = peer_addr(bar(Q_ACC_EMPTY + b), 0);
       const int ncols = n == 0 ? kFirstCols : BN;
 #pragma unroll 1
       for (int c0 = 0; c0 < ncols; c0 += 32) {
@@ -236,7 +292,7 @@ qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
       }
       if (n != 0) {
         tc_fence_before();
-        mbar_arrive(bar(Q_ACC_EMPTY + b));
+        mbar_arrive_cluster(empty_leader);
         continue;
       }
       // router: S slots of NP logits in columns [192, 256), added in order
@@ -245,7 +301,7 @@ qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
       tmem_ld32(acc + kFirstCols + 32, rs + 32);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(bar(Q_ACC_EMPTY + b));
+      mbar_arrive_cluster(empty_leader);
       float r[NP];
 #pragma unroll
       for (int mm = 0; mm < NP; ++mm) {
@@ -281,7 +337,7 @@ qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
         for (int mm = 0; mm < NP; ++mm) pr[mm] = 0.f;
       }
       // sum of p(i|x) over the warp's 32 tokens (one chunk row), fixed order
-      const int chunk = m * (BM / 32) + warp;
+      const int chunk = (m * 2 * BM + (int)rank * BM) / 32 + warp;
       if (chunk * 32 < p.N) {
         float* dst = p.partial + (size_t)chunk * p.M;
 #pragma unroll
@@ -297,10 +353,13 @@ qkv_route_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
     }
   }
 
+  // every product of the pair has completed (the leader drained them) and no
+  // remote arrival is pending before either CTA frees its TMEM and exits
   tc_fence_before();
   __syncthreads();
+  cluster_sync();
   tc_fence_after();
-  if (warp == 5) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512u) : "memory");
+  if (warp == 5) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512u) : "memory");
 }
 
 inline size_t router_bytes(int d) { return (size_t)kRouterCols * route_tc::dpad_of(d) * 2; }
@@ -308,16 +367,17 @@ inline size_t router_bytes(int d) { return (size_t)kRouterCols * route_tc::dpad_
 template <int NP>
 static moga_status launch_np(const Params& prm, const void* x, const void* w_qkv, const void* wx, int dpad,
                              cudaStream_t s) {
-  CUtensorMap mx, mw0, mw, mr;
+  CUtensorMap mx, mw128, mw64, mr;
   moga_status st;
   if ((st = route_tc::make_map(&mx, x, prm.N, prm.d, (int64_t)prm.d * 2, BM)) != MOGA_OK) return st;
-  if ((st = route_tc::make_map(&mw0, w_qkv, prm.n_out, prm.d, (int64_t)prm.d * 2, kFirstCols)) != MOGA_OK) return st;
-  if ((st = route_tc::make_map(&mw, w_qkv, prm.n_out, prm.d, (int64_t)prm.d * 2, BN)) != MOGA_OK) return st;
+  if ((st = route_tc::make_map(&mw128, w_qkv, prm.n_out, prm.d, (int64_t)prm.d * 2, BN / 2)) != MOGA_OK) return st;
+  if ((st = route_tc::make_map(&mw64, w_qkv, prm.n_out, prm.d, (int64_t)prm.d * 2, 64)) != MOGA_OK) return st;
   if ((st = route_tc::make_map(&mr, wx, kRouterCols, dpad, (int64_t)dpad * 2, kRouterCols)) != MOGA_OK) return st;
   cudaError_t e = cudaFuncSetAttribute(qkv_route_kernel<NP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return fail(MOGA_ERR_CUDA, "moga_qkv_route: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-  const int grid = std::min(prm.m_tiles * prm.n_tiles, route_tc::sm_count());
-  qkv_route_kernel<NP><<<grid, kThreads, kSmemBytes, s>>>(prm, mx, mw0, mw, mr);
+  // one pair of CTAs per pair of SMs (persistent), at most one pair per tile
+  const int pairs = std::min(prm.m_tiles * prm.n_tiles, route_tc::sm_count() / 2);
+  qkv_route_kernel<NP><<<2 * pairs, kThreads, kSmemBytes, s>>>(prm, mx, mw128, mw64, mr);
   return check_launch("moga_qkv_route");
 }
 
@@ -366,7 +426,7 @@ extern "C" moga_status moga_qkv_route(const void* x, const void* w_qkv, const vo
   prm.hhd = H * hd;
   prm.n_out = 3 * H * hd;
   prm.n_k = dpad / qkv::BK;
-  prm.m_tiles = ceil_div((int)N, qkv::BM);
+  prm.m_tiles = ceil_div((int)N, 2 * qkv::BM);   // 256-token tiles (one per SM pair)
   prm.n_tiles = 1 + ceil_div(prm.n_out - qkv::kFirstCols, qkv::BN);
   prm.bias = bias;
   prm.q = static_cast<__nv_bfloat16*>(q);
