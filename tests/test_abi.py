@@ -119,3 +119,51 @@ def test_mean_and_loss_argument_checks(lib):
 
 def test_version(lib):
     assert b"sm_100a" in lib.moga_version()
+
+
+def test_batch_sp_and_projection_workspace_sizes(lib):
+    assert lib.moga_permute_batched_ws_bytes(1000, 65, 16) == 0          # 1040 keys > 1024
+    assert lib.moga_permute_batched_ws_bytes(1000, 4, 5) == 2 * 2 * 20 * 4   # 2 tiles of 2048 tokens, 20 keys
+    assert lib.moga_qkv_route_ws_bytes(32760, 1536, 5) == 1024 * 5 * 4 + 64 * 1536 * 2
+    assert lib.moga_qkv_route_ws_bytes(32760, 12, 5) == 0                # d % 8
+    assert lib.moga_route_bwd_ws_bytes(100, 12, 4) == 0
+    assert lib.moga_attn_bwd_ws_bytes(1000, 2, 96) == 0                  # head_dim
+
+
+def test_batch_argument_checks(lib):
+    P = lib.moga_permute_batched
+    assert P(None, 100, 2, 4, FAKE, FAKE, FAKE, FAKE, FAKE, 4096, None) == 1
+    assert P(FAKE, 100, 0, 4, FAKE, FAKE, FAKE, FAKE, FAKE, 4096, None) == 1         # B
+    assert P(FAKE, 100, 2, 33, FAKE, FAKE, FAKE, FAKE, FAKE, 4096, None) == 1        # M
+    assert P(FAKE, 100, 65, 16, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 2    # too many keys
+    assert P(FAKE, 100, 2, 4, FAKE, FAKE, FAKE, FAKE, FAKE, 0, None) == 3            # workspace
+    W = 1 << 30
+    ga = lib.moga_group_attn_batched
+    assert ga(FAKE, FAKE, FAKE, 100, 0, 2, 128, FAKE, FAKE, 4, FAKE, 0.1, FAKE, None, FAKE, W, None) == 1
+    assert ga(FAKE, FAKE, FAKE, 100, 2, 2, 128, FAKE, FAKE, 40, FAKE, 0.1, FAKE, None, FAKE, W, None) == 1
+    assert lib.stga_attn_batched(FAKE, FAKE, FAKE, 0, 2, 128, None, 0.1, FAKE, FAKE, W, None) == 1
+    assert lib.moga_balance_loss_batched(FAKE, 3, FAKE, 100, 4, 0.1, FAKE, None) == 1   # N % B
+    assert lib.moga_balance_loss_batched(FAKE, 2, FAKE, 100, 0, 0.1, FAKE, None) == 1
+
+
+def test_sequence_parallel_argument_checks(lib):
+    assert lib.moga_sp_pack_heads(FAKE, 100, 12, 128, 5, FAKE, None) == 1      # 12 heads on 5 ranks
+    assert lib.moga_sp_unpack_heads(None, 100, 12, 128, 4, FAKE, None) == 1
+    mis = ctypes.c_void_p(4104)
+    assert lib.moga_sp_pack_heads(mis, 100, 12, 128, 4, FAKE, None) == 1       # alignment
+    assert lib.moga_balance_loss_part(FAKE, FAKE, 200, 100, 4, 0.1, FAKE, None) == 1   # n_local > N
+
+
+def test_projection_and_backward_argument_checks(lib):
+    q = lib.moga_qkv_route
+    W = 1 << 30
+    assert q(FAKE, FAKE, FAKE, None, 100, 12, 2, 128, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, W, None) == 1   # d % 8
+    assert q(FAKE, FAKE, FAKE, None, 100, 128, 2, 96, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, W, None) == 2   # head_dim
+    assert q(FAKE, FAKE, FAKE, None, 100, 128, 2, 128, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, None) == 3  # workspace
+    assert q(FAKE, FAKE, None, None, 100, 128, 2, 128, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, W, None) == 1
+    rb = lib.moga_route_bwd
+    assert rb(FAKE, FAKE, 1, 100, 12, 4, FAKE, FAKE, FAKE, FAKE, 0.1, 1.0, FAKE, FAKE, None, FAKE, W, None) == 1
+    assert rb(FAKE, FAKE, 1, 100, 16, 40, FAKE, FAKE, FAKE, FAKE, 0.1, 1.0, FAKE, FAKE, None, FAKE, W, None) == 1
+    gb = lib.moga_group_attn_bwd
+    assert gb(FAKE, FAKE, FAKE, 100, 2, 128, FAKE, FAKE, 4, FAKE, 0.1, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE,
+              FAKE, W, None) == 1   # null dout
