@@ -299,7 +299,7 @@ def run_ours(args):
         CALLS = ("route", "permute", "moga_group_attn", "stga_attn_mean", "moga_balance_loss")
     evl = [torch.cuda.Event(enable_timing=True) for _ in range(len(CALLS) + 1)]
 
-    def step(xd, qd, kd, vd, timed=False):
+    def step(xd, qd, kd, vd, timed=False, out=out, loss=loss):
         c = moga.check
 
         def mark(i):
@@ -364,13 +364,17 @@ def run_ours(args):
     job_ms = max_over_ranks(dev_ms, dev)
     value = job_throughput(world, N, args.steps, job_ms)
 
-    # ---- end to end through the public API: pinned host inputs in, result out
+    # ---- end to end through the C ABI: pinned host inputs in, result out
     hx, hq, hk, hv = (torch.from_numpy(inp[n].view(np.int16)).pin_memory() for n in ("x", "q", "k", "v"))
-    xd, qd, kd, vd = (torch.empty_like(a, device=dev) for a in (hx, hq, hk, hv))
+    hosts = (hx, hq, hk, hv)
     hout = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
     hloss = torch.empty(1, dtype=torch.float64).pin_memory()
-    h2d = sum(a.numel() * a.element_size() for a in (hx, hq, hk, hv))
+    h2d = sum(a.numel() * a.element_size() for a in hosts)
     d2h = hout.numel() * 2 + 8
+    bf = lambda t: t.view(torch.bfloat16)  # noqa: E731
+    # (a) serial: each step copies its inputs in, runs, and copies its result
+    # out on one stream
+    xd, qd, kd, vd = (torch.empty_like(a, device=dev) for a in hosts)
     e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
@@ -378,15 +382,59 @@ def run_ours(args):
     for i in range(args.steps):
         flush.zero_()
         e_evs[i][0].record(stream)
-        for dst, src in ((xd, hx), (qd, hq), (kd, hk), (vd, hv)):
+        for dst, src in zip((xd, qd, kd, vd), hosts):
             dst.copy_(src, non_blocking=True)
-        step(xd.view(torch.bfloat16), qd.view(torch.bfloat16), kd.view(torch.bfloat16), vd.view(torch.bfloat16))
+        step(bf(xd), bf(qd), bf(kd), bf(vd))
         hout.copy_(out, non_blocking=True)
         hloss.copy_(loss, non_blocking=True)
         e_evs[i][1].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e_evs)
-    e2e_value = job_throughput(world, N, args.steps, max_over_ranks(e2e_ms, dev))
+    serial_ms = sum(a.elapsed_time(b) for a, b in e_evs)
+    want_out, want_loss = hout.clone(), hloss.clone()
+    # (b) pipelined, as a stream of requests is served: step i's inputs go
+    # into buffer set i % 2 on a host-to-device stream and its result leaves
+    # output buffer i % 2 on a device-to-host stream, so the copies of one
+    # step overlap the kernels of its neighbours.  Every step's copies lie
+    # inside the timed region; its 400 MB of fresh inputs exceed L2.
+    ins = [(xd, qd, kd, vd), tuple(torch.empty_like(a, device=dev) for a in hosts)]
+    outs = [(out, loss), (torch.empty_like(out), torch.empty_like(loss))]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: [torch.cuda.Event() for _ in range(args.steps)]  # noqa: E731
+    copied, computed, returned = ev(), ev(), ev()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    s_in.wait_stream(stream)
+    for i in range(args.steps):
+        b = i & 1
+        if i >= 2:
+            s_in.wait_event(computed[i - 2])      # step i-2 has read buffer set b
+        with torch.cuda.stream(s_in):
+            for dst, src in zip(ins[b], hosts):
+                dst.copy_(src, non_blocking=True)
+        copied[i].record(s_in)
+        stream.wait_event(copied[i])
+        if i >= 2:
+            stream.wait_event(returned[i - 2])    # output buffer b has left
+        step(*(bf(t) for t in ins[b]), out=outs[b][0], loss=outs[b][1])
+        computed[i].record(stream)
+        s_out.wait_event(computed[i])
+        with torch.cuda.stream(s_out):
+            hout.copy_(outs[b][0], non_blocking=True)
+            hloss.copy_(outs[b][1], non_blocking=True)
+        returned[i].record(s_out)
+    stream.wait_event(returned[-1])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    pipe_ms = t0.elapsed_time(t1)
+    moga.device_status()
+    # the last step's result crossed the streams intact
+    if not (torch.equal(hout, want_out) and torch.equal(hloss, want_loss)):
+        raise RuntimeError("pipelined end-to-end result differs from the serial one")
+    e2e_value = job_throughput(world, N, args.steps, max_over_ranks(pipe_ms, dev))
+    e2e_serial = job_throughput(world, N, args.steps, max_over_ranks(serial_ms, dev))
 
     counts_h = counts.cpu().numpy()
     fl_moga = moga_flops(counts_h, H, hd)
@@ -411,7 +459,9 @@ def run_ours(args):
         "stga_tflops": fl_stga / (statistics.median(call_ms[CALLS[3]]) / 1000.0) / 1e12,
         "mean_fused_into_stga": bool(args.fused_mean),
         "route_permute_hbm": route_permute_hbm(wl, call_ms, pk),
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "pipelined": True, "ms_per_step": pipe_ms / args.steps, "serial_value": e2e_serial,
+                "serial_ms_per_step": serial_ms / args.steps},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
