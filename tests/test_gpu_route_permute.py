@@ -89,3 +89,24 @@ def test_skewed_router_fraction(cuda_device):
     case = Case(W.MULTISHOT_10S, with_qkv=False)
     g, _, _ = case.route64()
     assert 0.395 <= np.mean(g == 0) <= 0.405
+
+
+@pytest.mark.parametrize("N,M,skew", [(1, 1, 0.0), (31, 5, 0.0), (33, 32, 0.0), (1024, 5, 0.9), (32760, 32, 0.0),
+                                      (65535, 5, 0.6), (65536, 32, 0.0), (65537, 5, 0.0), (100000, 32, 0.99),
+                                      (65536, 1, 0.0)])
+def test_permute_sizes_bit_exact(N, M, skew, cuda_device):
+    """The permute on random ids, a share `skew` of them in group 0, from one
+    token to several 2048-token tiles with ragged tails and up to 32 groups:
+    bit-exact against the oracle."""
+    import torch
+    import sparse_attention_long_moga_b200 as moga
+    rs = np.random.default_rng(N + M)
+    g = rs.integers(0, M, N).astype(np.int32)
+    g[rs.random(N) < skew] = 0
+    perm, cu, counts, mx = moga.moga_permute(torch.from_numpy(g).to(cuda_device), M)
+    moga.device_status()
+    rp, rcu, rcounts, rmx = opermute.permute(g, M)
+    assert np.array_equal(perm.cpu().numpy(), rp.astype(np.int32))
+    assert np.array_equal(cu.cpu().numpy(), rcu.astype(np.int32))
+    assert np.array_equal(counts.cpu().numpy(), rcounts.astype(np.int32))
+    assert int(mx.item()) == rmx
