@@ -346,8 +346,10 @@ moga_status moga_balance_loss_batched(const int32_t* counts, int32_t B, const vo
  * ws:     moga_qkv_route_ws_bytes(N, d, M) bytes, 256-byte aligned; on
  *         return it starts with the per-32-token sums of p(i|x) that
  *         moga_balance_loss reads, in moga_route's layout.
- * Requires d % 8 == 0, hd in {64, 128}, 1 <= M <= 32, 16-byte aligned x,
- * w_qkv, q, k, v. */
+ * Requires d % 8 == 0, 1 <= M <= 32, 16-byte aligned x, w_qkv, q, k, v
+ * (else MOGA_ERR_INVALID_ARG) and hd in {64, 128} (else
+ * MOGA_ERR_UNSUPPORTED); a smaller workspace returns MOGA_ERR_WORKSPACE.
+ * moga_qkv_route_ws_bytes returns 0 for arguments the call rejects. */
 size_t moga_qkv_route_ws_bytes(int64_t N, int32_t d, int32_t M);
 moga_status moga_qkv_route(const void* x, const void* w_qkv, const void* w_r, const float* bias, int64_t N,
                            int32_t d, int32_t H, int32_t hd, int32_t M, void* q, void* k, void* v,
