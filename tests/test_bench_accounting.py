@@ -1,0 +1,53 @@
+"""The work the benchmark divides by (its roofline `achieved` and the layer
+TFLOP/s) against a count made independently from the oracle's own groups.
+
+Attention FLOPs are 4 * H * hd per visible (query, key) pair.  The benchmark
+counts the static branches from the geometry in closed form (run lengths,
+borrowed frames per side, windows per frame) and MoGA from the group counts;
+here the same totals come from enumerating every window group, frame group
+and routed group the oracle builds and summing n_q * n_kv, or, for MoGA on a
+small case, from the dense same-group mask.
+"""
+import numpy as np
+import pytest
+
+import bench
+from oracle import permute as opermute
+from oracle import stga as ostga
+from synth import workloads as W
+
+CASES = [
+    W.TINY,
+    W.WAN13B_5S,
+    W.MULTISHOT_10S,
+    # a middle shot shorter than the borrowed-frame count, temporal groups of 2
+    W.Workload("acct_short_shot", T=5, h=6, w=10, d=64, H=3, hd=128, M=7, shots=(2, 1, 2), tg_max=2, win_h=3,
+               win_w=5),
+    # several runs per shot, ragged run lengths, four shots
+    W.Workload("acct_runs", T=23, h=8, w=8, d=64, H=2, hd=64, M=4, shots=(7, 5, 9, 2), tg_max=3, win_h=4,
+               win_w=4, aug=3),
+]
+
+
+@pytest.mark.parametrize("wl", CASES, ids=lambda w: w.name)
+def test_stga_flops_equal_enumerated_groups(wl):
+    geom = W.stga_shape(wl)
+    pairs = sum(len(q) * len(kv) for q, kv in ostga.window_groups(geom))
+    pairs += sum(len(q) * len(kv) for q, kv in ostga.frame_groups(geom))
+    assert bench.stga_flops(wl) == 4.0 * wl.H * wl.hd * pairs
+
+
+def test_stga_flops_of_the_bench_workload():
+    # window groups: 4 windows x 3 runs of 7 frames x (7 * 390)^2; frames: 21 x 1560^2
+    wl = W.WAN13B_5S
+    assert bench.stga_flops(wl) == 4.0 * 12 * 128 * (4 * 3 * (7 * 390) ** 2 + 21 * 1560 ** 2)
+
+
+@pytest.mark.parametrize("N,M", [(1, 1), (300, 7), (2000, 5)])
+def test_moga_flops_equal_dense_mask(N, M):
+    rs = np.random.default_rng(N * 31 + M)
+    g = rs.integers(0, M, N)
+    g[rs.random(N) < 0.3] = 0
+    counts = opermute.permute(g, M)[2]
+    pairs = int(np.count_nonzero(g[:, None] == g[None, :]))
+    assert bench.moga_flops(counts, 3, 64) == 4.0 * 3 * 64 * pairs
