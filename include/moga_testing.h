@@ -10,15 +10,25 @@
  *   the device error word, drains its in-flight copies, frees its tensor
  *   memory and exits (no trap, no hang).  moga_device_status() reports it.
  * Pass (0, 0) to restore normal operation.
+ *
+ * moga_test_stga_groups(geom, out, cap) validates geom as stga_attn does and
+ * returns the number n of temporal groups its launches use (-1 if stga_attn
+ * would reject the geometry; moga_last_error() says why), writing for group
+ * i < min(n, cap) the four int32 values out[4i .. 4i+3] = (first frame, end
+ * frame (exclusive), frames borrowed from the previous shot, frames borrowed
+ * from the next shot).  Host code only: no device is touched.
  */
 #ifndef MOGA_TESTING_H
 #define MOGA_TESTING_H
+
+#include "moga.h"
 
 #ifdef __cplusplus
 extern "C" {
 #endif
 
 void moga_test_set_attn_debug(long long timeout_cycles, int flags);
+int32_t moga_test_stga_groups(const moga_stga_geom* geom, int32_t* out, int32_t cap);
 
 #ifdef __cplusplus
 }

@@ -40,6 +40,7 @@
 
 #include "common.cuh"
 #include "tc_common.cuh"
+#include "../../include/moga_testing.h"
 
 namespace moga {
 namespace attn {
@@ -965,6 +966,24 @@ extern "C" moga_status stga_attn_mean(const void* q, const void* k, const void* 
   if (!out) return fail(MOGA_ERR_INVALID_ARG, "stga_attn_mean: null out");
   return stga_impl(q, k, v, H, hd, geom, softmax_scale, o_acc, o_acc, nullptr, nullptr, false, out, ws, ws_bytes,
                    stream, "stga_attn_mean");
+}
+
+// Test hook (declared in include/moga_testing.h): the temporal groups the
+// static-group launches use for a geometry, as (first frame, end frame,
+// borrowed frames before, borrowed frames after) per group, in time order.
+// Host code only: it validates the geometry exactly as stga_attn does and
+// launches nothing.
+extern "C" int32_t moga_test_stga_groups(const moga_stga_geom* geom, int32_t* out, int32_t cap) {
+  Params prm;
+  int64_t N = 0;
+  if (stga_params(geom, 1, 1.0f, prm, N, "moga_test_stga_groups") != MOGA_OK) return -1;
+  for (int i = 0; i < prm.n_tg && i < cap; ++i) {
+    out[4 * i + 0] = prm.tg[i].t0;
+    out[4 * i + 1] = prm.tg[i].t1;
+    out[4 * i + 2] = prm.tg[i].a_prev;
+    out[4 * i + 3] = prm.tg[i].a_next;
+  }
+  return prm.n_tg;
 }
 
 extern "C" moga_status stga_attn_train(const void* q, const void* k, const void* v, int32_t H, int32_t hd,
