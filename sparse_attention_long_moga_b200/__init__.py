@@ -37,29 +37,55 @@ def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
-def _need(t, dtype, name, dim=None):
-    if not t.is_cuda:
-        raise ValueError("%s must be a CUDA tensor" % name)
+def _need(t, dtype, name, dim=None, shape=None, device=True):
+    """Type, rank, shape and layout (the library sees only pointers, so a short
+    buffer would be read past its end), then, unless device=False (the caller
+    checks all its tensors' residence at once with _on_device after their
+    shapes), residence on the current CUDA device."""
     if t.dtype != dtype:
         raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
-    if not t.is_contiguous():
-        raise ValueError("%s must be contiguous" % name)
     if dim is not None and t.dim() != dim:
         raise ValueError("%s must have %d dims" % (name, dim))
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if device:
+        _on_device(**{name: t})
+
+
+def _on_device(**tensors):
+    """Every tensor on the current CUDA device (the calls launch on its current stream)."""
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("%s must be a CUDA tensor" % name)
+        if t.device.index != torch.cuda.current_device():
+            raise ValueError("%s is on %s but the calls run on the current device cuda:%d"
+                             % (name, t.device, torch.cuda.current_device()))
+
+
+def _check_geom(geom: dict, N: int):
+    """stga_attn takes the token count from the geometry: it must match q's rows."""
+    n = geom["T"] * geom["h"] * geom["w"]
+    if n != N:
+        raise ValueError("geometry has T*h*w = %d tokens but q, k, v have %d rows" % (n, N))
 
 
 def moga_route(x: torch.Tensor, w_r: torch.Tensor, bias: torch.Tensor | None = None):
     """r = x W_r (+bias), p = softmax(r), g = argmax p.  Returns (g int32 [N], gate fp32 [N], ws)."""
     if x.dtype not in (torch.float32, torch.bfloat16):
         raise ValueError("x must be float32 or bfloat16")
-    _need(x, x.dtype, "x", 2)
-    _need(w_r, x.dtype, "w_r", 2)
+    _need(x, x.dtype, "x", 2, device=False)
+    _need(w_r, x.dtype, "w_r", 2, device=False)
     N, d = x.shape
     M = w_r.shape[1]
     if w_r.shape[0] != d:
         raise ValueError("w_r must be [d, M]")
     if bias is not None:
-        _need(bias, torch.float32, "bias", 1)
+        _need(bias, torch.float32, "bias", 1, (M,), device=False)
+    _on_device(x=x, w_r=w_r, bias=bias)
     L = lib()
     ws_bytes = L.moga_route_ws_bytes(N, d, M)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=x.device)
@@ -75,15 +101,16 @@ def moga_qkv_route(x: torch.Tensor, w_qkv: torch.Tensor, w_r: torch.Tensor, bias
                    hd: int):
     """The Q/K/V projection with the router fused in: x [N, d] bf16, w_qkv [3*H*hd, d] bf16
     (a linear layer's weight), w_r [d, M] bf16.  Returns (q, k, v [N, H, hd] bf16, g, gate, ws)."""
-    _need(x, torch.bfloat16, "x", 2)
-    _need(w_qkv, torch.bfloat16, "w_qkv", 2)
-    _need(w_r, torch.bfloat16, "w_r", 2)
+    _need(x, torch.bfloat16, "x", 2, device=False)
+    _need(w_qkv, torch.bfloat16, "w_qkv", 2, device=False)
+    _need(w_r, torch.bfloat16, "w_r", 2, device=False)
     N, d = x.shape
     M = w_r.shape[1]
     if w_qkv.shape != (3 * H * hd, d) or w_r.shape[0] != d:
         raise ValueError("w_qkv must be [3*H*hd, d] and w_r [d, M]")
     if bias is not None:
-        _need(bias, torch.float32, "bias", 1)
+        _need(bias, torch.float32, "bias", 1, (M,), device=False)
+    _on_device(x=x, w_qkv=w_qkv, w_r=w_r, bias=bias)
     L = lib()
     ws = torch.empty(max(L.moga_qkv_route_ws_bytes(N, d, M), 16), dtype=torch.uint8, device=x.device)
     q, k, v = (torch.empty((N, H, hd), dtype=torch.bfloat16, device=x.device) for _ in range(3))
@@ -111,11 +138,13 @@ def moga_permute(group_id: torch.Tensor, M: int):
     return perm, cu, counts, mx
 
 
-def _check_qkv(q, k, v):
+def _check_qkv(q, k, v, device=True):
     for name, t in (("q", q), ("k", k), ("v", v)):
-        _need(t, torch.bfloat16, name, 3)
+        _need(t, torch.bfloat16, name, 3, device=False)
     if not (q.shape == k.shape == v.shape):
         raise ValueError("q, k, v must share the shape [N, H, hd]")
+    if device:
+        _on_device(q=q, k=k, v=v)
     return q.shape
 
 
@@ -131,13 +160,15 @@ def attn_workspace(q: torch.Tensor) -> torch.Tensor:
 def moga_group_attn(q, k, v, perm, cu_seqlens, gate_prob, M: int, softmax_scale: float | None = None,
                     o_acc: torch.Tensor | None = None, ws: torch.Tensor | None = None):
     """o_acc[perm[j]] = gate * softmax(q k^T * scale) v inside each group (written, fp32)."""
-    N, H, hd = _check_qkv(q, k, v)
-    _need(perm, torch.int32, "perm", 1)
-    _need(cu_seqlens, torch.int32, "cu_seqlens", 1)
-    _need(gate_prob, torch.float32, "gate_prob", 1)
+    N, H, hd = _check_qkv(q, k, v, device=False)
+    _need(perm, torch.int32, "perm", 1, (N,), device=False)
+    _need(cu_seqlens, torch.int32, "cu_seqlens", 1, (M + 1,), device=False)
+    _need(gate_prob, torch.float32, "gate_prob", 1, (N,), device=False)
+    if o_acc is not None:
+        _need(o_acc, torch.float32, "o_acc", 3, (N, H, hd), device=False)
+    _on_device(q=q, k=k, v=v, perm=perm, cu_seqlens=cu_seqlens, gate_prob=gate_prob, o_acc=o_acc, ws=ws)
     if o_acc is None:
         o_acc = torch.empty((N, H, hd), dtype=torch.float32, device=q.device)
-    _need(o_acc, torch.float32, "o_acc", 3)
     scale = 1.0 / math.sqrt(hd) if softmax_scale is None else softmax_scale
     ws = attn_workspace(q) if ws is None else ws
     check(lib().moga_group_attn(_ptr(q), _ptr(k), _ptr(v), N, H, hd, _ptr(perm), _ptr(cu_seqlens), M,
@@ -157,10 +188,13 @@ def geom_struct(geom: dict):
 def stga_attn(q, k, v, geom: dict, softmax_scale: float | None = None, o_acc: torch.Tensor | None = None,
               ws: torch.Tensor | None = None):
     """o_acc += window-group attention + per-frame attention (fp32)."""
-    N, H, hd = _check_qkv(q, k, v)
+    N, H, hd = _check_qkv(q, k, v, device=False)
+    _check_geom(geom, N)
+    if o_acc is not None:
+        _need(o_acc, torch.float32, "o_acc", 3, (N, H, hd), device=False)
+    _on_device(q=q, k=k, v=v, o_acc=o_acc, ws=ws)
     if o_acc is None:
         o_acc = torch.zeros((N, H, hd), dtype=torch.float32, device=q.device)
-    _need(o_acc, torch.float32, "o_acc", 3)
     scale = 1.0 / math.sqrt(hd) if softmax_scale is None else softmax_scale
     s, keep = geom_struct(geom)
     ws = attn_workspace(q) if ws is None else ws
@@ -173,11 +207,14 @@ def stga_attn(q, k, v, geom: dict, softmax_scale: float | None = None, o_acc: to
 def stga_attn_mean(q, k, v, geom: dict, o_acc: torch.Tensor, softmax_scale: float | None = None,
                    out: torch.Tensor | None = None, ws: torch.Tensor | None = None):
     """out = bf16((o_acc + window-group attention + per-frame attention) / 3), mean fused into the frame pass."""
-    N, H, hd = _check_qkv(q, k, v)
-    _need(o_acc, torch.float32, "o_acc", 3)
+    N, H, hd = _check_qkv(q, k, v, device=False)
+    _check_geom(geom, N)
+    _need(o_acc, torch.float32, "o_acc", 3, (N, H, hd), device=False)
+    if out is not None:
+        _need(out, torch.bfloat16, "out", 3, (N, H, hd), device=False)
+    _on_device(q=q, k=k, v=v, o_acc=o_acc, out=out, ws=ws)
     if out is None:
         out = torch.empty((N, H, hd), dtype=torch.bfloat16, device=q.device)
-    _need(out, torch.bfloat16, "out", 3)
     scale = 1.0 / math.sqrt(hd) if softmax_scale is None else softmax_scale
     s, keep = geom_struct(geom)
     ws = attn_workspace(q) if ws is None else ws
@@ -189,17 +226,26 @@ def stga_attn_mean(q, k, v, geom: dict, o_acc: torch.Tensor, softmax_scale: floa
 
 def visual_attn_mean(o_acc: torch.Tensor, out: torch.Tensor | None = None):
     """out = bf16(o_acc / 3)."""
-    _need(o_acc, torch.float32, "o_acc")
+    _need(o_acc, torch.float32, "o_acc", device=False)
+    if out is not None:
+        _need(out, torch.bfloat16, "out", shape=o_acc.shape, device=False)
+    _on_device(o_acc=o_acc, out=out)
     if out is None:
         out = torch.empty(o_acc.shape, dtype=torch.bfloat16, device=o_acc.device)
-    _need(out, torch.bfloat16, "out")
     check(lib().visual_attn_mean(_ptr(o_acc), o_acc.numel(), _ptr(out), _stream()), "visual_attn_mean")
     return out
 
 
 def moga_balance_loss(counts, route_ws, N: int, M: int, alpha: float, loss: torch.Tensor | None = None):
     """L_gb = alpha * M * sum_i F_i P_i as a fp64 device scalar."""
-    _need(counts, torch.int32, "counts", 1)
+    _need(counts, torch.int32, "counts", 1, (M,), device=False)
+    _need(route_ws, torch.uint8, "route_ws", 1, device=False)
+    if route_ws.numel() < 4 * M * -(-N // 32):
+        raise ValueError("route_ws holds %d bytes, fewer than the router's per-32-token sums for N=%d, M=%d"
+                         % (route_ws.numel(), N, M))
+    if loss is not None:
+        _need(loss, torch.float64, "loss", 1, (1,), device=False)
+    _on_device(counts=counts, route_ws=route_ws, loss=loss)
     if loss is None:
         loss = torch.empty(1, dtype=torch.float64, device=counts.device)
     check(lib().moga_balance_loss(_ptr(counts), _ptr(route_ws), N, M, alpha, _ptr(loss), _stream()),
@@ -218,6 +264,9 @@ def visual_attention_forward(x, w_r, bias, q, k, v, M: int, geom: dict, alpha: f
 
     fused_mean=True takes the mean inside the STGA frame pass (stga_attn_mean);
     False runs stga_attn then visual_attn_mean."""
+    if x.dim() != 2 or q.dim() != 3 or x.shape[0] != q.shape[0]:
+        raise ValueError("x must be [N, d] and q, k, v [N, H, hd] with the same N")
+    _check_geom(geom, q.shape[0])
     g, gate, ws = moga_route(x, w_r, bias)
     perm, cu, counts, mx = moga_permute(g, M)
     ws_attn = attn_workspace(q)
@@ -270,6 +319,7 @@ def visual_attention_forward_batched(x, w_r, bias, q, k, v, M: int, geom: dict, 
     if q.shape[:2] != (B, N) or k.shape != q.shape or v.shape != q.shape:
         raise ValueError("q, k, v must be [B, N, H, hd] with x's B and N")
     H, hd = q.shape[2], q.shape[3]
+    _check_geom(geom, N)
     qf, kf, vf = (t.reshape(B * N, H, hd) for t in (q, k, v))
     g, gate, rws = moga_route(x.reshape(B * N, d), w_r, bias)
     perm, cu, counts, mx = moga_permute_batched(g, B, M)
@@ -301,7 +351,14 @@ def visual_attention_forward_train(x, w_r, bias, q, k, v, M: int, geom: dict, al
     """Forward that saves what the backward needs.  Returns dict(out, loss, saved)."""
     L = lib()
     N, d = x.shape
-    _, H, hd = _check_qkv(q, k, v)
+    Nq, H, hd = _check_qkv(q, k, v)
+    if Nq != N:
+        raise ValueError("x has %d rows, q, k, v %d" % (N, Nq))
+    _check_geom(geom, N)
+    _need(x, x.dtype, "x", 2)
+    _need(w_r, x.dtype, "w_r", 2, (d, M))
+    if bias is not None:
+        _need(bias, torch.float32, "bias", 1, (M,))
     dev = x.device
     scale = 1.0 / math.sqrt(hd) if softmax_scale is None else softmax_scale
     rws = torch.empty(max(L.moga_route_ws_bytes(N, d, M), 16), dtype=torch.uint8, device=dev)
@@ -341,8 +398,11 @@ def visual_attention_backward(saved: dict, x, w_r, q, k, v, M: int, geom: dict, 
     dbias [M] fp32 or None, dgate [N] fp32)."""
     L = lib()
     N, d = x.shape
-    _, H, hd = _check_qkv(q, k, v)
-    _need(dout, torch.bfloat16, "dout", 3)
+    Nq, H, hd = _check_qkv(q, k, v)
+    if Nq != N:
+        raise ValueError("x has %d rows, q, k, v %d" % (N, Nq))
+    _check_geom(geom, N)
+    _need(dout, torch.bfloat16, "dout", 3, (N, H, hd))
     dev = q.device
     f32 = dict(dtype=torch.float32, device=dev)
     dq, dk, dv = (torch.zeros((N, H, hd), **f32) for _ in range(3))
