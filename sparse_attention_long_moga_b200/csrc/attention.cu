@@ -668,8 +668,7 @@ static moga_status make_map(CUtensorMap* m, const void* base, int64_t rows, int 
 }
 
 static long long default_timeout_cycles() {
-  // about two seconds at the maximum SM clock
-  return 4000000000LL;
+  return kWaitLimitCycles;
 }
 
 template <int HD>

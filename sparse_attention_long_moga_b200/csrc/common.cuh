@@ -25,4 +25,9 @@ __device__ __forceinline__ void record_device_error(int code) {
 
 __host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Limit of every bounded wait on an mbarrier, in SM clock cycles: about two
+// seconds at the maximum SM clock.  A wait that runs out records
+// MOGA_ERR_TIMEOUT in the device error word and the kernel returns.
+constexpr long long kWaitLimitCycles = 4000000000LL;
+
 }  // namespace moga

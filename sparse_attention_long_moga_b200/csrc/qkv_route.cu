@@ -390,6 +390,6 @@ extern "C" moga_status moga_qkv_route(const void* x, const void* w_qkv, const vo
   prm.group_id = group_id;
   prm.gate_prob = gate_prob;
   prm.partial = static_cast<float*>(ws);
-  prm.timeout = 4000000000LL;
+  prm.timeout = kWaitLimitCycles;
   return NP == 16 ? qkv::launch_np<16>(prm, x, w_qkv, wx, dpad, s) : qkv::launch_np<32>(prm, x, w_qkv, wx, dpad, s);
 }

@@ -272,7 +272,7 @@ static moga_status route_impl(const void* x, const void* w_r, moga_dtype dt, con
   if (dt == MOGA_BF16) {
     // tensor-core path; W_r^T scratch after the partial rows
     void* wt = static_cast<uint8_t*>(ws) + route_partial_bytes(N, M);
-    return route_tc::launch(x, w_r, bias, (int)N, d, M, group_id, gate_prob, partial, probs, wt, 4000000000LL, s);
+    return route_tc::launch(x, w_r, bias, (int)N, d, M, group_id, gate_prob, partial, probs, wt, kWaitLimitCycles, s);
   }
   return route_detail::dispatch<float>(x, w_r, bias, (int)N, d, M, group_id, gate_prob, partial, probs, s);
 }

@@ -28,7 +28,7 @@
 namespace moga {
 namespace route_bwd_detail {
 
-constexpr long long kTimeoutCycles = 4000000000LL;   // about two seconds at the maximum SM clock
+constexpr long long kTimeoutCycles = kWaitLimitCycles;
 
 constexpr int kDrThreads = 256;   // route_dr_kernel: tokens per block
 constexpr int kThreads = 128;     // route_bwd_kernel: threads per block
