@@ -340,6 +340,27 @@ def visual_attention_forward_batched(x, w_r, bias, q, k, v, M: int, geom: dict, 
     return dict(out=out, loss=loss, g=g, gate=gate, perm=perm, cu_seqlens=cu, counts=counts, max_seqlen=mx)
 
 
+def _check_layer_args(x, w_r, q, k, v, M: int, geom: dict, bias=None, dout=None):
+    """Shapes of the training calls' inputs, then their residence: x [N, d]
+    (fp32 or bf16) and w_r [d, M] of x's dtype, q/k/v [N, H, hd] bf16, bias
+    [M] fp32, dout [N, H, hd] bf16, a geometry of N tokens."""
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("x must be float32 or bfloat16")
+    _need(x, x.dtype, "x", 2, device=False)
+    N, d = x.shape
+    _need(w_r, x.dtype, "w_r", 2, (d, M), device=False)
+    Nq, H, hd = _check_qkv(q, k, v, device=False)
+    if Nq != N:
+        raise ValueError("x has %d rows, q, k, v %d" % (N, Nq))
+    _check_geom(geom, N)
+    if bias is not None:
+        _need(bias, torch.float32, "bias", 1, (M,), device=False)
+    if dout is not None:
+        _need(dout, torch.bfloat16, "dout", 3, (N, H, hd), device=False)
+    _on_device(x=x, w_r=w_r, q=q, k=k, v=v, bias=bias, dout=dout)
+    return N, d, H, hd
+
+
 # ---------------------------------------------------------------- training
 #
 # The training forward keeps the router probabilities, the three branch
@@ -350,15 +371,7 @@ def visual_attention_forward_train(x, w_r, bias, q, k, v, M: int, geom: dict, al
                                    softmax_scale: float | None = None):
     """Forward that saves what the backward needs.  Returns dict(out, loss, saved)."""
     L = lib()
-    N, d = x.shape
-    Nq, H, hd = _check_qkv(q, k, v)
-    if Nq != N:
-        raise ValueError("x has %d rows, q, k, v %d" % (N, Nq))
-    _check_geom(geom, N)
-    _need(x, x.dtype, "x", 2)
-    _need(w_r, x.dtype, "w_r", 2, (d, M))
-    if bias is not None:
-        _need(bias, torch.float32, "bias", 1, (M,))
+    N, d, H, hd = _check_layer_args(x, w_r, q, k, v, M, geom, bias=bias)
     dev = x.device
     scale = 1.0 / math.sqrt(hd) if softmax_scale is None else softmax_scale
     rws = torch.empty(max(L.moga_route_ws_bytes(N, d, M), 16), dtype=torch.uint8, device=dev)
@@ -397,12 +410,7 @@ def visual_attention_backward(saved: dict, x, w_r, q, k, v, M: int, geom: dict, 
     Returns dict(dq, dk, dv [N, H, hd] fp32, dx [N, d] fp32, dw_r [d, M] fp32,
     dbias [M] fp32 or None, dgate [N] fp32)."""
     L = lib()
-    N, d = x.shape
-    Nq, H, hd = _check_qkv(q, k, v)
-    if Nq != N:
-        raise ValueError("x has %d rows, q, k, v %d" % (N, Nq))
-    _check_geom(geom, N)
-    _need(dout, torch.bfloat16, "dout", 3, (N, H, hd))
+    N, d, H, hd = _check_layer_args(x, w_r, q, k, v, M, geom, dout=dout)
     dev = q.device
     f32 = dict(dtype=torch.float32, device=dev)
     dq, dk, dv = (torch.zeros((N, H, hd), **f32) for _ in range(3))

@@ -90,3 +90,26 @@ def test_router_and_layer_shapes():
     wq = torch.zeros((3 * H * HD, 64), dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="w_qkv must be"):
         moga.moga_qkv_route(x, wq[:-1], w, None, H, HD)
+
+
+def test_training_call_shapes():
+    x = torch.zeros((N, 64), dtype=torch.bfloat16)
+    w = torch.zeros((64, M), dtype=torch.bfloat16)
+    q, k, v = _qkv()
+    dout = torch.zeros((N, H, HD), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        moga.visual_attention_forward_train(x, w, None, q, k, v, M, GEOM, 0.1)
+    with pytest.raises(ValueError, match="w_r must be torch.bfloat16"):
+        moga.visual_attention_forward_train(x, w.float(), None, q, k, v, M, GEOM, 0.1)
+    with pytest.raises(ValueError, match="w_r must have shape"):
+        moga.visual_attention_forward_train(x, w[:, :-1], None, q, k, v, M, GEOM, 0.1)
+    with pytest.raises(ValueError, match="bias must have shape"):
+        moga.visual_attention_forward_train(x, w, _f32(M - 1), q, k, v, M, GEOM, 0.1)
+    with pytest.raises(ValueError, match="rows"):
+        moga.visual_attention_forward_train(x[:-32], w, None, q, k, v, M, GEOM, 0.1)
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        moga.visual_attention_backward({}, x, w, q, k, v, M, GEOM, 0.1, dout, 1.0)
+    with pytest.raises(ValueError, match="dout must have shape"):
+        moga.visual_attention_backward({}, x, w, q, k, v, M, GEOM, 0.1, dout[:-1], 1.0)
+    with pytest.raises(ValueError, match="geometry has"):
+        moga.visual_attention_backward({}, x, w, q, k, v, M, dict(GEOM, T=3, shots=[3]), 0.1, dout, 1.0)
