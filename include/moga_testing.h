@@ -17,6 +17,18 @@
  * i < min(n, cap) the four int32 values out[4i .. 4i+3] = (first frame, end
  * frame (exclusive), frames borrowed from the previous shot, frames borrowed
  * from the next shot).  Host code only: no device is touched.
+ *
+ * moga_test_attn_tiles(mode, cu_seqlens, M, N, H, geom, out, cap) returns the
+ * number n of work tiles one attention launch processes (-1 on invalid
+ * arguments) and writes for tile L < min(n, cap), in launch order, the five
+ * int32 values out[5L .. 5L+4] = (head, query begin, query end, key begin,
+ * key end), rows in the launch's index space: segment order for mode 0
+ * (MoGA; cu_seqlens is a HOST array of M+1 entries, N tokens), the
+ * window-major order for mode 1 (windows; geom), token order for mode 2
+ * (frames; geom).  moga_test_window_tokens(geom, begin, end, out) writes the
+ * tokens at window-major positions [begin, end) to out and returns their
+ * count (-1 on invalid arguments).  Both run the kernels' own index code
+ * compiled for the host; no device is touched.
  */
 #ifndef MOGA_TESTING_H
 #define MOGA_TESTING_H
@@ -29,6 +41,9 @@ extern "C" {
 
 void moga_test_set_attn_debug(long long timeout_cycles, int flags);
 int32_t moga_test_stga_groups(const moga_stga_geom* geom, int32_t* out, int32_t cap);
+int32_t moga_test_attn_tiles(int32_t mode, const int32_t* cu_seqlens, int32_t M, int64_t N, int32_t H,
+                             const moga_stga_geom* geom, int32_t* out, int32_t cap);
+int32_t moga_test_window_tokens(const moga_stga_geom* geom, int32_t begin, int32_t end, int32_t* out);
 
 #ifdef __cplusplus
 }

@@ -114,10 +114,20 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 // ------------------------------------------------------------------ index maps
 
+// Read-only load: through the non-coherent cache on the device; a plain load
+// when the same index code runs on the host (test hooks).
+__host__ __device__ __forceinline__ int load_ro(const int32_t* a) {
+#ifdef __CUDA_ARCH__
+  return __ldg(a);
+#else
+  return *a;
+#endif
+}
+
 // Token at position idx of the window-major order (window, frame, position
 // inside the window), in which a temporal group's keys/values -- including
 // the frames borrowed from the neighbouring shots -- are one contiguous range.
-__device__ __forceinline__ int window_token(const Params& p, int idx) {
+__host__ __device__ __forceinline__ int window_token(const Params& p, int idx) {
   const int local = idx % p.whw;
   const int wf = idx / p.whw;
   const int frame = wf % p.T;
@@ -148,10 +158,10 @@ struct GroupTable {
 
 // unit_rows: query rows per work unit (two 128-row tiles in the forward, one
 // in the backward)
-__device__ void build_group_table(const Params& p, GroupTable& gt, int unit_rows = 2 * BM) {
+__host__ __device__ void build_group_table(const Params& p, GroupTable& gt, int unit_rows = 2 * BM) {
   int size[32], order[32];
   for (int i = 0; i < p.M; ++i) {
-    size[i] = __ldg(p.cu + i + 1) - __ldg(p.cu + i);
+    size[i] = load_ro(p.cu + i + 1) - load_ro(p.cu + i);
     order[i] = i;
   }
   for (int i = 1; i < p.M; ++i) {   // insertion sort, descending size, stable
@@ -167,7 +177,7 @@ __device__ void build_group_table(const Params& p, GroupTable& gt, int unit_rows
   gt.prefix[0] = 0;
   for (int k = 0; k < p.M; ++k) {
     const int g = order[k];
-    gt.start[k] = __ldg(p.cu + g);
+    gt.start[k] = load_ro(p.cu + g);
     gt.size[k] = size[g];
     gt.prefix[k + 1] = gt.prefix[k] + ceil_div(size[g], unit_rows) * p.H;
   }
@@ -175,7 +185,7 @@ __device__ void build_group_table(const Params& p, GroupTable& gt, int unit_rows
 
 // Tile L (a pair of 128-row query tiles of one group and head).  Tiles are
 // ordered so that consecutive ones share a group's K/V through L2.
-__device__ __forceinline__ Tile decode_tile(const Params& p, const GroupTable& gt, int L) {
+__host__ __device__ __forceinline__ Tile decode_tile(const Params& p, const GroupTable& gt, int L) {
   Tile t;
   t.valid = 0;
   constexpr int kPair = 2 * BM;
@@ -983,6 +993,62 @@ extern "C" int32_t moga_test_stga_groups(const moga_stga_geom* geom, int32_t* ou
     out[4 * i + 3] = prm.tg[i].a_next;
   }
   return prm.n_tg;
+}
+
+// Test hooks (include/moga_testing.h): the work tiles of one attention launch
+// and the window-major token order, computed by the kernels' own index code
+// (decode_tile, build_group_table, window_token) compiled for the host.
+extern "C" int32_t moga_test_attn_tiles(int32_t mode, const int32_t* cu_seqlens, int32_t M, int64_t N, int32_t H,
+                                        const moga_stga_geom* geom, int32_t* out, int32_t cap) {
+  Params prm;
+  if (mode == MODE_MOGA) {
+    if (!cu_seqlens || M < 1 || M > 32 || N <= 0 || N > INT32_MAX || H <= 0) {
+      fail(MOGA_ERR_INVALID_ARG, "moga_test_attn_tiles: bad MoGA arguments");
+      return -1;
+    }
+    memset(&prm, 0, sizeof(prm));
+    prm.N = (int)N;
+    prm.H = H;
+    prm.M = M;
+    prm.cu = cu_seqlens;
+  } else if (mode == MODE_WINDOW || mode == MODE_FRAME) {
+    int64_t n = 0;
+    if (stga_params(geom, H, 1.0f, prm, n, "moga_test_attn_tiles") != MOGA_OK) return -1;
+  } else {
+    fail(MOGA_ERR_INVALID_ARG, "moga_test_attn_tiles: mode %d", mode);
+    return -1;
+  }
+  prm.mode = mode;
+  GroupTable gt;
+  memset(&gt, 0, sizeof(gt));
+  if (mode == MODE_MOGA) build_group_table(prm, gt);
+  int32_t n = 0;
+  for (int L = 0;; ++L) {
+    const Tile t = decode_tile(prm, gt, L);
+    if (!t.valid) break;
+    if (n < cap) {
+      int32_t* o = out + 5 * (size_t)n;
+      o[0] = t.head;
+      o[1] = t.q_begin;
+      o[2] = t.q_end;
+      o[3] = t.kv_begin;
+      o[4] = t.kv_end;
+    }
+    ++n;
+  }
+  return n;
+}
+
+extern "C" int32_t moga_test_window_tokens(const moga_stga_geom* geom, int32_t begin, int32_t end, int32_t* out) {
+  Params prm;
+  int64_t N = 0;
+  if (stga_params(geom, 1, 1.0f, prm, N, "moga_test_window_tokens") != MOGA_OK) return -1;
+  if (begin < 0 || end > N || begin > end) {
+    fail(MOGA_ERR_INVALID_ARG, "moga_test_window_tokens: range [%d, %d) outside [0, %lld)", begin, end, (long long)N);
+    return -1;
+  }
+  for (int i = begin; i < end; ++i) out[i - begin] = window_token(prm, i);
+  return end - begin;
 }
 
 extern "C" moga_status stga_attn_train(const void* q, const void* k, const void* v, int32_t H, int32_t hd,
