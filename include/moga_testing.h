@@ -29,6 +29,15 @@
  * tokens at window-major positions [begin, end) to out and returns their
  * count (-1 on invalid arguments).  Both run the kernels' own index code
  * compiled for the host; no device is touched.
+ *
+ * moga_test_bwd_units(mode, keys, cu_seqlens, M, N, H, geom, grid, out, cap)
+ * does the same for the backward: *grid receives the number of CTAs the
+ * launch uses (the dQ kernel for keys = 0, the dK/dV kernel for keys = 1),
+ * the return value is the number n of valid units among them (-1 on invalid
+ * arguments), and unit i < min(n, cap) is written as the seven int32 values
+ * out[7i .. 7i+6] = (head, query begin, query end, key begin, key end, tile
+ * begin, tile end), the tile being a range of queries (keys = 0) or of keys
+ * (keys = 1) of at most 128 rows.
  */
 #ifndef MOGA_TESTING_H
 #define MOGA_TESTING_H
@@ -44,6 +53,8 @@ int32_t moga_test_stga_groups(const moga_stga_geom* geom, int32_t* out, int32_t 
 int32_t moga_test_attn_tiles(int32_t mode, const int32_t* cu_seqlens, int32_t M, int64_t N, int32_t H,
                              const moga_stga_geom* geom, int32_t* out, int32_t cap);
 int32_t moga_test_window_tokens(const moga_stga_geom* geom, int32_t begin, int32_t end, int32_t* out);
+int32_t moga_test_bwd_units(int32_t mode, int32_t keys, const int32_t* cu_seqlens, int32_t M, int64_t N,
+                            int32_t H, const moga_stga_geom* geom, int32_t* grid, int32_t* out, int32_t cap);
 
 #ifdef __cplusplus
 }

@@ -64,7 +64,7 @@ struct Unit {
 
 // KEYS: tile over the key range (dK/dV) instead of the query range (dQ).
 template <bool KEYS>
-__device__ __forceinline__ Unit decode_unit(const BwdParams& b, const GroupTable& gt, int L) {
+__host__ __device__ __forceinline__ Unit decode_unit(const BwdParams& b, const GroupTable& gt, int L) {
   const Params& p = b.f;
   Unit u;
   u.valid = 0;
@@ -809,6 +809,30 @@ extern "C" size_t moga_attn_bwd_ws_bytes(int64_t N, int32_t H, int32_t hd) {
   return moga::attn::bwd_ws_bytes(N, H, hd);
 }
 
+namespace moga {
+namespace attn {
+
+// Units launched for the MoGA branch: an upper bound on the 128-row tiles of
+// all groups (sum of ceil(n_i / 128) <= N / 128 + M per head); units past the
+// last tile exit at once.
+static int moga_bwd_units(int64_t N, int M, int H) { return (ceil_div((int)N, BM) + M) * H; }
+
+// Window branch: prefixes of the 128-query-tile and 128-key-tile units over
+// the temporal groups (windows x heads x tiles per group).
+static void fill_window_units(BwdParams& b, int H) {
+  const Params& p = b.f;
+  b.q_units[0] = b.kv_units[0] = 0;
+  for (int i = 0; i < p.n_tg; ++i) {
+    const TGroup& tg = p.tg[i];
+    const int qlen = (tg.t1 - tg.t0) * p.whw, kvlen = (tg.t1 - tg.t0 + tg.a_prev + tg.a_next) * p.whw;
+    b.q_units[i + 1] = b.q_units[i] + p.n_win * H * ceil_div(qlen, BM);
+    b.kv_units[i + 1] = b.kv_units[i] + p.n_win * H * ceil_div(kvlen, BM);
+  }
+}
+
+}  // namespace attn
+}  // namespace moga
+
 extern "C" moga_status moga_group_attn_bwd(const void* q, const void* k, const void* v, int64_t N, int32_t H,
                                            int32_t hd, const int32_t* perm, const int32_t* cu_seqlens, int32_t M,
                                            const float* gate_prob, float softmax_scale, const float* o_moga,
@@ -838,8 +862,7 @@ extern "C" moga_status moga_group_attn_bwd(const void* q, const void* k, const v
   b.dq = dq;
   b.dk = dk;
   b.dv = dv;
-  // upper bound on the 128-row tiles of all groups: N / 128 + M per head
-  const int units = (ceil_div((int)N, BM) + M) * H;
+  const int units = moga_bwd_units(N, M, H);
   return run_branch_bwd(b, hd, units, units, q, k, v, dout, o_moga, lse, dgate, ws,
                         static_cast<cudaStream_t>(stream));
 }
@@ -866,13 +889,7 @@ extern "C" moga_status stga_attn_bwd(const void* q, const void* k, const void* v
   b.dk = dk;
   b.dv = dv;
   const Params& p = b.f;
-  b.q_units[0] = b.kv_units[0] = 0;
-  for (int i = 0; i < p.n_tg; ++i) {
-    const TGroup& tg = p.tg[i];
-    const int qlen = (tg.t1 - tg.t0) * p.whw, kvlen = (tg.t1 - tg.t0 + tg.a_prev + tg.a_next) * p.whw;
-    b.q_units[i + 1] = b.q_units[i] + p.n_win * H * ceil_div(qlen, BM);
-    b.kv_units[i + 1] = b.kv_units[i] + p.n_win * H * ceil_div(kvlen, BM);
-  }
+  fill_window_units(b, H);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   b.f.mode = MODE_WINDOW;
   if ((st = run_branch_bwd(b, hd, b.q_units[p.n_tg], b.kv_units[p.n_tg], q, k, v, dout, o_win, lse_win, nullptr, ws,
@@ -881,4 +898,60 @@ extern "C" moga_status stga_attn_bwd(const void* q, const void* k, const void* v
   b.f.mode = MODE_FRAME;
   const int fu = p.T * H * ceil_div(p.hw, BM);
   return run_branch_bwd(b, hd, fu, fu, q, k, v, dout, o_frame, lse_frame, nullptr, ws, s);
+}
+
+// Test hook (include/moga_testing.h): the work units of one backward launch
+// (keys = 0: the dQ kernel, tiles over queries; keys = 1: the dK/dV kernel,
+// tiles over keys), decoded by the kernels' own decode_unit compiled for the
+// host, with the grid the launch uses.  Host code only.
+extern "C" int32_t moga_test_bwd_units(int32_t mode, int32_t keys, const int32_t* cu_seqlens, int32_t M, int64_t N,
+                                       int32_t H, const moga_stga_geom* geom, int32_t* grid, int32_t* out,
+                                       int32_t cap) {
+  using namespace moga;
+  using namespace moga::attn;
+  BwdParams b;
+  memset(&b, 0, sizeof(b));
+  int g = 0;
+  if (mode == MODE_MOGA) {
+    if (!cu_seqlens || M < 1 || M > 32 || N <= 0 || N > INT32_MAX || H <= 0) {
+      fail(MOGA_ERR_INVALID_ARG, "moga_test_bwd_units: bad MoGA arguments");
+      return -1;
+    }
+    b.f.N = (int)N;
+    b.f.H = H;
+    b.f.M = M;
+    b.f.cu = cu_seqlens;
+    g = moga_bwd_units(N, M, H);
+  } else if (mode == MODE_WINDOW || mode == MODE_FRAME) {
+    int64_t n = 0;
+    if (stga_params(geom, H, 1.0f, b.f, n, "moga_test_bwd_units") != MOGA_OK) return -1;
+    fill_window_units(b, H);
+    g = mode == MODE_WINDOW ? (keys ? b.kv_units[b.f.n_tg] : b.q_units[b.f.n_tg])
+                            : b.f.T * H * ceil_div(b.f.hw, BM);
+  } else {
+    fail(MOGA_ERR_INVALID_ARG, "moga_test_bwd_units: mode %d", mode);
+    return -1;
+  }
+  b.f.mode = mode;
+  GroupTable gt;
+  memset(&gt, 0, sizeof(gt));
+  if (mode == MODE_MOGA) build_group_table(b.f, gt, BM);
+  if (grid) *grid = g;
+  int32_t n = 0;
+  for (int L = 0; L < g; ++L) {
+    const Unit u = keys ? decode_unit<true>(b, gt, L) : decode_unit<false>(b, gt, L);
+    if (!u.valid) continue;
+    if (n < cap) {
+      int32_t* o = out + 7 * (size_t)n;
+      o[0] = u.head;
+      o[1] = u.q_begin;
+      o[2] = u.q_end;
+      o[3] = u.kv_begin;
+      o[4] = u.kv_end;
+      o[5] = u.t_begin;
+      o[6] = u.t_end;
+    }
+    ++n;
+  }
+  return n;
 }

@@ -156,3 +156,95 @@ def test_hook_rejections(hooks):
     out = (ctypes.c_int32 * 8)()
     assert wtok(ctypes.byref(g), 0, 9, out) == -1
     assert wtok(ctypes.byref(g), 0, 8, out) == 8
+
+
+@pytest.fixture(scope="module")
+def bwd_hook(hooks):
+    lib = _lib.load()
+    fn = lib.moga_test_bwd_units
+    fn.restype = ctypes.c_int32
+    fn.argtypes = [ctypes.c_int32, ctypes.c_int32, I32P, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32,
+                   ctypes.POINTER(_lib.StgaGeom), I32P, I32P, ctypes.c_int32]
+    return fn, hooks[1]
+
+
+def _units(fn, mode, keys, H, cu=None, N=0, geom=None):
+    cu_arr = None if cu is None else (ctypes.c_int32 * len(cu))(*[int(c) for c in cu])
+    g = keep = None
+    if geom is not None:
+        g, keep = _geom(geom)
+    grid = ctypes.c_int32(0)
+    args = (mode, keys, cu_arr, 0 if cu is None else len(cu) - 1, N, H, None if g is None else ctypes.byref(g),
+            ctypes.byref(grid))
+    n = fn(*args, None, 0)
+    assert n >= 0
+    out = (ctypes.c_int32 * (7 * max(n, 1)))()
+    assert fn(*args, out, n) == n
+    del keep
+    return grid.value, np.frombuffer(out, dtype=np.int32)[:7 * n].reshape(n, 7)
+
+
+@settings(max_examples=100, deadline=None)
+@given(st.lists(st.integers(0, 700), min_size=1, max_size=32), st.integers(1, 3), st.booleans())
+def test_moga_backward_units_cover_every_row_once(bwd_hook, sizes, H, keys):
+    fn, _ = bwd_hook
+    N = sum(sizes)
+    if N == 0:
+        return
+    cu = np.concatenate([[0], np.cumsum(sizes)])
+    grid, units = _units(fn, 0, int(keys), H, cu=cu, N=N)
+    assert len(units) <= grid       # the launch's upper-bound grid reaches every tile
+    cover = np.zeros((H, N), dtype=np.int64)
+    seg = {(int(cu[i]), int(cu[i + 1])) for i in range(len(sizes)) if sizes[i]}
+    for h, q0, q1, k0, k1, t0, t1 in units:
+        assert (q0, q1) == (k0, k1) and (q0, q1) in seg
+        assert q0 <= t0 < t1 <= q1 and t1 - t0 <= 128 and (t0 - q0) % 128 == 0
+        cover[h, t0:t1] += 1
+    assert np.all(cover == 1)
+
+
+@settings(max_examples=80, deadline=None)
+@given(geometries(), st.integers(1, 3))
+def test_static_backward_units_match_oracle_groups(bwd_hook, geom, H):
+    fn, wtok = bwd_hook
+    hw = geom["h"] * geom["w"]
+    N = geom["T"] * hw
+    for keys in (0, 1):
+        grid, units = _units(fn, 2, keys, H, geom=geom)
+        assert len(units) == grid
+        cover = np.zeros((H, N), dtype=np.int64)
+        for h, q0, q1, k0, k1, t0, t1 in units:
+            assert (q0, q1) == (k0, k1) and q0 % hw == 0 and q1 == q0 + hw and t1 - t0 <= 128
+            cover[h, t0:t1] += 1
+        assert np.all(cover == 1)
+    order = _window_tokens(wtok, geom, N)
+    groups = ostga.window_groups(geom)
+    group_of = np.empty(N, dtype=np.int64)      # two groups may share their keys, never a query
+    for i, (q, _) in enumerate(groups):
+        group_of[q] = i
+    # dQ: every (head, token) is a query of exactly one unit
+    grid, units = _units(fn, 1, 0, H, geom=geom)
+    assert len(units) == grid
+    cover = np.zeros((H, N), dtype=np.int64)
+    for h, q0, q1, k0, k1, t0, t1 in units:
+        gi = group_of[order[q0]]
+        assert np.array_equal(order[q0:q1], groups[gi][0]) and np.array_equal(order[k0:k1], groups[gi][1])
+        assert q0 <= t0 < t1 <= q1 and t1 - t0 <= 128
+        cover[h, order[t0:t1]] += 1
+    assert np.all(cover == 1)
+    # dK/dV: every key of every (group, head) in exactly one unit
+    grid, units = _units(fn, 1, 1, H, geom=geom)
+    assert len(units) == grid
+    seen = {}
+    for h, q0, q1, k0, k1, t0, t1 in units:
+        gi = group_of[order[q0]]
+        assert np.array_equal(order[q0:q1], groups[gi][0]) and np.array_equal(order[k0:k1], groups[gi][1])
+        assert k0 <= t0 < t1 <= k1 and t1 - t0 <= 128
+        seen.setdefault((gi, int(h)), []).append((int(t0 - k0), int(t1 - k0)))
+    assert len(seen) == len(groups) * H
+    for (gi, h), parts in seen.items():
+        n_kv = len(groups[gi][1])
+        c = np.zeros(n_kv, dtype=np.int64)
+        for a, b in parts:
+            c[a:b] += 1
+        assert np.all(c == 1)
