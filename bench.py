@@ -1,17 +1,20 @@
 #!/usr/bin/env python
 """Benchmark: MoGA visual-attention layer forward (route, permute, MoGA group
 attention, STGA window + frame attention, three-way mean, balance loss) on
-synthetic Wan-1.3B-shaped latents: 21 frames x 30 x 52 = 32,760 tokens,
-d = 1536, 12 heads x 128, M = 5, one shot, temporal groups of <= 7 frames,
-15 x 26 windows.
+synthetic Wan-shaped latents.  Default workload: the 60 s ten-shot video at
+24 fps, 361 frames x 30 x 52 = 563,160 tokens, d = 5120, 40 heads x 128,
+M = 20, router input drawn from 20 Gaussian clusters, temporal groups of
+<= 7 frames, 15 x 26 windows, two borrowed frames per side at each cut.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload NAME]
 
 One step = one full layer forward over one sequence, inputs resident in HBM.
 Between timed steps a 256 MiB buffer is written to flush L2 (outside the
 timed events).  Under torchrun each rank runs its own sequence (independent
 problems, no data-path collective); the job time is the max over ranks.
 `--impl reference` times the fp64 CPU oracle on a bounded sample instead.
+`--workload` picks another workload of the suite (each gives its own line).
 """
 from __future__ import annotations
 
@@ -33,17 +36,34 @@ import numpy as np  # noqa: E402
 from synth import workloads as W  # noqa: E402
 
 METRIC = "visual-attn layer fwd tokens/s (bf16); group-attn % of tcgen05 bf16 peak"
-WORKLOAD = W.WAN13B_5S
+# the headline workload: the largest single-GPU configuration of the suite
+HEADLINE = W.LONG_60S
+# the training, batch, sequence-parallel and projection modes default to the 5 s workload
+SECONDARY = W.WAN13B_5S
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
 # DRAM bytes (read + write) of one moga_group_attn call on the 5 s Wan-1.3B
-# workload, from an ncu --set full capture of this bench command:
+# workload (32,760 tokens x 12 heads x 128), from an ncu --set full capture:
 # gather3_kernel<0> 302.1 + 263.1 MB, attn_kernel<128> (MoGA launch)
 # 305.1 + 162.2 MB.  Set to None whenever either kernel changes, until it is
 # captured again.
 CALL_TRAFFIC_BYTES = 1.0325e9
+CALL_TRAFFIC_UNITS = 32760 * 12 * 128
 CALL_TRAFFIC_SOURCE = "ncu dram__bytes_read.sum + dram__bytes_write.sum, gather3_kernel<0> + attn_kernel<128> MoGA launch"
+
+
+def call_traffic(wl):
+    """DRAM bytes of one moga_group_attn call: the captured figure, scaled by
+    the Q/K/V elements processed for another workload (the copy moves every
+    element once and each group's K/V stays L2-resident while its tiles run)."""
+    if CALL_TRAFFIC_BYTES is None:
+        return None, "not captured for the current kernels"
+    units = wl.N * wl.H * wl.hd
+    if units == CALL_TRAFFIC_UNITS:
+        return CALL_TRAFFIC_BYTES, CALL_TRAFFIC_SOURCE + " (captured on this workload)"
+    return CALL_TRAFFIC_BYTES * units / CALL_TRAFFIC_UNITS, (
+        CALL_TRAFFIC_SOURCE + ", captured on the 32,760-token workload and scaled by N*H*hd")
 
 
 def peaks():
@@ -58,15 +78,21 @@ def peaks():
 def route_permute_hbm(wl, call_ms, pk):
     """Algorithmic bytes of the router (x once, g and gate out, one Σp row per 32 tokens)
     and of the permute (g in, perm out; counts and cu are negligible) over their
-    CUDA-event call times, as a fraction of the measured HBM copy bandwidth."""
+    CUDA-event call times, as a fraction of the measured HBM copy bandwidth; also
+    the two calls as one unit (bytes of both over the sum of their times)."""
     xb = 2 if wl.x_dtype == "bf16" else 4
     route_b = wl.N * wl.d * xb + 8 * wl.N + 4 * wl.M * (-(-wl.N // 32))
     perm_b = 8 * wl.N + 8 * (wl.M + 1)
     out = {}
+    tot_b, tot_ms = 0, 0.0
     for name, b in (("route", route_b), ("permute", perm_b)):
         ms = statistics.median(call_ms[name])
         gbs = b / (ms * 1e-3) / 1e9
         out[name] = {"bytes": b, "ms": ms, "gbs": gbs, "frac": gbs / pk["hbm_gbs"]}
+        tot_b += b
+        tot_ms += ms
+    gbs = tot_b / (tot_ms * 1e-3) / 1e9
+    out["unit"] = {"bytes": tot_b, "ms": tot_ms, "gbs": gbs, "frac": gbs / pk["hbm_gbs"]}
     return out
 
 
@@ -171,70 +197,131 @@ def make_inputs(wl):
 
 # ----------------------------------------------------------------------------- CPU oracle arm
 
-def oracle_sample(wl, inputs, heads=(0,)):
-    """Times the fp64 oracle as it stands: route + permute + loss over all N
-    tokens, then the MoGA, window and frame attention and the mean over all N
-    tokens for the listed heads.  Returns (tokens/s extrapolated to all heads,
-    details)."""
-    from oracle import attention as oatt
+ROUTE_CHUNK = 16384
+
+
+def _f64(a):
+    return W.bf16_bits_to_f64(a) if a.dtype == np.uint16 else a.astype(np.float64)
+
+
+def oracle_sample(wl, inputs, seed=1, n_heads=8, per_head=512):
+    """Times the fp64 oracle as it stands on a bounded sample of one layer forward.
+
+    Route over all N tokens (in row chunks of ROUTE_CHUNK, one after another),
+    permute and loss over all N; then, for n_heads heads spread over [0, H),
+    the three attention branches and the mean at a stratified sample of
+    per_head tokens (every MoGA group, window group, both sides of every cut
+    and every frame), each row computed from its full definition.  The
+    attention time is extrapolated to the whole layer by the exact per-row
+    cost (keys per row over the three branches, summed over all tokens and
+    heads); the per-head widening of q, k, v to float64 is timed apart and
+    scaled by heads.  Returns (tokens/s, details)."""
     from oracle import layer as olayer
     from oracle import permute as opermute
     from oracle import route as oroute
+    from oracle import sample as osample
     from oracle import stga as ostga
 
-    x = W.bf16_bits_to_f64(inputs["x"]) if inputs["x"].dtype == np.uint16 else inputs["x"].astype(np.float64)
-    w = W.bf16_bits_to_f64(inputs["w_r"]) if inputs["w_r"].dtype == np.uint16 else inputs["w_r"].astype(np.float64)
+    N, H = wl.N, wl.H
+    w = _f64(inputs["w_r"])
     t0 = time.perf_counter()
-    g, p_g, p = oroute.route(x, w, W.bias_f64(wl))
-    perm, cu, counts, mx = opermute.permute(g, wl.M)
+    g = np.empty(N, dtype=np.int64)
+    p_g = np.empty(N)
+    p = np.empty((N, wl.M))
+    for a in range(0, N, ROUTE_CHUNK):
+        b = min(a + ROUTE_CHUNK, N)
+        g[a:b], p_g[a:b], p[a:b] = oroute.route(_f64(inputs["x"][a:b]), w, W.bias_f64(wl))
+    perm, cu, counts, _ = opermute.permute(g, wl.M)
     olayer.balance_loss(counts, p, wl.alpha)
     t_route = time.perf_counter() - t0
 
     geom = W.stga_shape(wl)
     scale = 1.0 / math.sqrt(wl.hd)
-    t_attn = 0.0
-    for h in heads:
-        qh, kh, vh = (W.bf16_bits_to_f64(inputs[n][:, h:h + 1, :]) for n in ("q", "k", "v"))
+    rows = osample.stratified_rows(geom, g, wl.M, H, n_heads=n_heads, per_head=per_head, seed=seed)
+    # keys per row over the three branches, for every token
+    kv_moga = counts[g]
+    kv_win = np.zeros(N, dtype=np.int64)
+    for qt, kvt in ostga.window_groups(geom):
+        kv_win[qt] = len(kvt)
+    cost_tok = kv_moga + kv_win + wl.hw
+    t_conv = t_rows = t_mean = 0.0
+    n_rows = 0
+    cost_sample = 0.0
+    for h, toks in rows.items():
         t0 = time.perf_counter()
-        om = oatt.moga(qh, kh, vh, g, p_g, wl.M, scale)
-        ow = oatt.grouped(qh, kh, vh, ostga.window_groups(geom), scale)
-        of = oatt.grouped(qh, kh, vh, ostga.frame_groups(geom), scale)
+        qh, kh, vh = (W.bf16_bits_to_f64(inputs[n][:, h, :]) for n in ("q", "k", "v"))
+        t_conv += time.perf_counter() - t0
+        t0 = time.perf_counter()
+        om, ow, of = osample.branch_rows(qh, kh, vh, toks, g, p_g, wl.M, geom, scale)
+        t_rows += time.perf_counter() - t0
+        t0 = time.perf_counter()
         olayer.mean3(om, ow, of)
-        t_attn += time.perf_counter() - t0
-    t_layer = t_route + t_attn * (wl.H / len(heads))
-    return wl.N / t_layer, dict(t_route_s=t_route, t_attn_s=t_attn, heads=len(heads))
+        t_mean += time.perf_counter() - t0
+        n_rows += len(toks)
+        cost_sample += float(cost_tok[toks].sum())
+    cost_total = float(cost_tok.sum()) * H
+    t_attn = t_conv / len(rows) * H + t_rows * cost_total / cost_sample
+    t_mean_all = t_mean * (N * H) / n_rows
+    t_layer = t_route + t_attn + t_mean_all
+    return N / t_layer, dict(t_route_s=t_route, t_conv_s=t_conv, t_rows_s=t_rows, t_mean_s=t_mean,
+                             heads=len(rows), rows=n_rows, t_layer_extrapolated_s=t_layer)
 
 
-def cpu_threads():
+def oracle_sample_text(wl, det):
+    return ("fp64 oracle, extrapolated: route+permute+loss over all %d tokens (%.1f s); attention (MoGA, window, "
+            "frame) + mean at a stratified sample of %d (token, head) rows over %d of %d heads covering every "
+            "group, window group, cut side and frame (%.1f s rows + %.1f s widening), scaled by exact per-row "
+            "key counts to all %d x %d rows -> %.0f s per layer"
+            % (wl.N, det["t_route_s"], det["rows"], det["heads"], wl.H, det["t_rows_s"], det["t_conv_s"], wl.N,
+               wl.H, det["t_layer_extrapolated_s"]))
+
+
+def host_cores():
+    """(cpus the host offers, BLAS threads numpy's matmul uses)."""
+    blas = None
     try:
         from threadpoolctl import threadpool_info
         n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
+        blas = max(n) if n else None
     except Exception:
-        return os.cpu_count() or 1
+        blas = None
+    try:
+        avail = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        avail = os.cpu_count() or 1
+    return avail, (blas if blas is not None else 1)
+
+
+def cpu_baseline_dict(wl, value, det):
+    avail, blas = host_cores()
+    return {"value": value, "unit": "tokens/s", "cores": blas, "host_cpus": avail, "blas_threads": blas,
+            "kind": "oracle", "sample": oracle_sample_text(wl, det)}
+
+
+def pick_workload(args, default):
+    """The suite workload named by --workload (its stored skew bias filled in), else `default`."""
+    return W.resolved(W.SUITE[args.workload] if args.workload else default)
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    wl = WORKLOAD
+    wl = pick_workload(args, HEADLINE)
     inputs = make_inputs(wl)
     for i in range(args.warmup):
-        oracle_sample(wl, inputs, heads=(i % wl.H,))
+        oracle_sample(wl, inputs, seed=100 + i, n_heads=2, per_head=256)
     t0 = time.perf_counter()
-    vals = [oracle_sample(wl, inputs, heads=(s % wl.H,))[0] for s in range(args.steps)]
+    # 4 heads per step keeps a 10-step run within a few minutes on a few host cores
+    res = [oracle_sample(wl, inputs, seed=1 + s, n_heads=4) for s in range(args.steps)]
     el = time.perf_counter() - t0
-    value = float(statistics.median(vals))
-    sample = ("fp64 oracle per step: route+permute+loss over all %d tokens, attention (MoGA+window+frame+mean) "
-              "over all tokens for 1 of %d heads, extrapolated to all heads" % (wl.N, wl.H))
+    value = float(statistics.median([r[0] for r in res]))
+    det = res[len(res) // 2][1]
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * el / max(args.steps, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic",
-            "config": dict(config_dict(wl), l2="n/a (host cores)", parallelism="fp64 oracle on the host cores"),
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
-                             "sample": sample},
+            "data": "synthetic", "config": config_dict(wl),
+            "cpu_baseline": cpu_baseline_dict(wl, value, det),
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -243,8 +330,17 @@ def run_reference(args):
 def config_dict(wl):
     return {"workload": wl.name, "tokens": wl.N, "frames": wl.T, "grid": [wl.h, wl.w], "d": wl.d,
             "heads": wl.H, "head_dim": wl.hd, "M": wl.M, "shots": list(wl.shots), "tg_max": wl.tg_max,
-            "window": [wl.win_h, wl.win_w], "aug_frames": wl.aug, "sequences_per_gpu": 1,
-            "l2": "flushed between timed steps (256 MiB write)", "parallelism": "independent sequences per GPU"}
+            "window": [wl.win_h, wl.win_w], "aug_frames": wl.aug, "router": router_kind(wl),
+            "sequences_per_gpu": 1, "l2": "flushed between timed steps (256 MiB write); inputs exceed L2",
+            "parallelism": "independent sequences per GPU"}
+
+
+def router_kind(wl):
+    if wl.clusters:
+        return "clustered input (%d Gaussian centres)" % wl.clusters
+    if wl.bias0 is not None:
+        return "skewed (bias on group 0)"
+    return "i.i.d. input"
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -263,7 +359,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     import sparse_attention_long_moga_b200 as moga
-    wl = WORKLOAD
+    wl = pick_workload(args, HEADLINE)
     inp = make_inputs(wl)
     geom = W.stga_shape(wl)
 
@@ -273,6 +369,9 @@ def run_ours(args):
 
     x, w_r, q, k, v = (to_dev(inp[n]) for n in ("x", "w_r", "q", "k", "v"))
     N, M, H, hd = wl.N, wl.M, wl.H, wl.hd
+    bias = None
+    if wl.bias0 is not None:
+        bias = torch.from_numpy(W.bias_f64(wl).astype(np.float32)).to(dev)
     L = moga._lib.lib()
     stream = torch.cuda.current_stream()
     sp = moga._stream()
@@ -307,8 +406,8 @@ def run_ours(args):
             if timed:
                 evl[i].record(stream)
         mark(0)
-        c(L.moga_route(P(xd), P(w_r), moga.MOGA_BF16, None, N, wl.d, M, P(g), P(gate), P(rws), rws.numel(), sp),
-          "route")
+        c(L.moga_route(P(xd), P(w_r), moga.MOGA_BF16, P(bias) if bias is not None else None, N, wl.d, M, P(g),
+                       P(gate), P(rws), rws.numel(), sp), "route")
         mark(1)
         c(L.moga_permute(P(g), N, M, P(perm), P(cu), P(counts), P(mx), P(pws), pws.numel(), sp), "permute")
         mark(2)
@@ -443,6 +542,11 @@ def run_ours(args):
     pk, pk_kind = peaks()
     moga_avg_s = statistics.mean(moga_ms) / 1000.0
     achieved = fl_moga / moga_avg_s / 1e12
+    # a kernel timed inside a timed region of seconds runs under the power
+    # cap: the sustained peak applies; a short region gets the burst peak
+    sustained = job_ms > 1000.0
+    peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
+    traffic, traffic_src = call_traffic(wl)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": job_ms / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -450,14 +554,17 @@ def run_ours(args):
         "config": config_dict(wl),
         "roofline": {"bound": "tensor",
                      "kernel": "moga_group_attn call = gather3_kernel (segment-order copy) + attn_kernel<128>",
-                     "achieved": achieved,
-                     "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
-                     "peak_kind": "%s burst dense bf16" % pk_kind, "traffic": CALL_TRAFFIC_BYTES,
-                     "traffic_source": CALL_TRAFFIC_SOURCE,
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_kind": "%s %s dense bf16" % (pk_kind, "sustained" if sustained else "burst"),
+                     "frac_of_burst": achieved / pk["bf16_tflops"],
+                     "traffic": traffic, "traffic_source": traffic_src,
                      "flops_per_launch": fl_moga, "launch_ms": moga_avg_s * 1e3},
         "layer_tflops": (fl_moga + fl_stga) / (job_ms / args.steps / 1000.0) / 1e12,
         "breakdown_ms": {name: statistics.median(v) for name, v in call_ms.items()},
         "stga_tflops": fl_stga / (statistics.median(call_ms[CALLS[3]]) / 1000.0) / 1e12,
+        "stga_frac": fl_stga / (statistics.median(call_ms[CALLS[3]]) / 1000.0) / 1e12 / peak,
+        "group_sizes": {"min": int(counts_h.min()), "max": int(counts_h.max()), "sum_sq": float(np.sum(
+            counts_h.astype(np.float64) ** 2))},
         "mean_fused_into_stga": bool(args.fused_mean),
         "route_permute_hbm": route_permute_hbm(wl, call_ms, pk),
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -467,11 +574,8 @@ def run_ours(args):
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu_val, det = oracle_sample(wl, inp, heads=(0, 1))
-        line["cpu_baseline"] = {"value": cpu_val, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
-                                "sample": "fp64 oracle: route+permute+loss over all %d tokens, attention+mean over "
-                                          "all tokens for 2 of %d heads, extrapolated to all heads (%.1f s route, "
-                                          "%.1f s attention)" % (N, H, det["t_route_s"], det["t_attn_s"])}
+        cpu_val, det = oracle_sample(wl, inp)
+        line["cpu_baseline"] = cpu_baseline_dict(wl, cpu_val, det)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -490,7 +594,7 @@ def run_train(args):
     import sparse_attention_long_moga_b200 as moga
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(0)
-    wl = WORKLOAD
+    wl = pick_workload(args, SECONDARY)
     inp = make_inputs(wl)
     geom = W.stga_shape(wl)
 
@@ -616,7 +720,7 @@ def run_batch(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(0)
     B = args.batch
-    per = WORKLOAD.with_(M=20)
+    per = pick_workload(args, SECONDARY).with_(M=20)
     big = per.with_(name="%s_x%d" % (per.name, B), T=per.T * B, shots=tuple(per.shots) * B)
     inp = make_inputs(big)
     geom = W.stga_shape(per)
@@ -717,7 +821,7 @@ def run_sp(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     import sparse_attention_long_moga_b200 as moga
     from sparse_attention_long_moga_b200.sp import sp_visual_attention_forward
-    wl = WORKLOAD
+    wl = pick_workload(args, SECONDARY)
     if wl.H % world or wl.N % world:
         if rank == 0:
             print(json.dumps({"metric": "visual-attn layer fwd tokens/s, sequence-parallel (bf16)",
@@ -786,7 +890,7 @@ def run_qkv(args):
     import sparse_attention_long_moga_b200 as moga
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(0)
-    wl = WORKLOAD
+    wl = pick_workload(args, SECONDARY)
     inp = make_inputs(wl)
     x = torch.from_numpy(inp["x"].view(np.int16)).to(dev).view(torch.bfloat16)
     w_r = torch.from_numpy(inp["w_r"].view(np.int16)).to(dev).view(torch.bfloat16)
@@ -851,9 +955,12 @@ def run_qkv(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(W.SUITE), default=None,
+                    help="suite workload (default: %s for the forward, %s for the other modes)"
+                    % (HEADLINE.name, SECONDARY.name))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fused-mean", action="store_true",
                     help="run stga_attn_mean (mean inside the STGA frame pass) instead of stga_attn + visual_attn_mean")

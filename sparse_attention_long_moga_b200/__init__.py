@@ -24,9 +24,9 @@ import torch
 
 from ._lib import MOGA_BF16, MOGA_F32, MogaError, StgaGeom, check, lib  # noqa: F401
 
-__all__ = ["moga_route", "moga_permute", "moga_group_attn", "stga_attn", "stga_attn_mean", "visual_attn_mean",
-           "moga_balance_loss", "visual_attention_forward", "attn_workspace", "device_status", "MogaError", "geom_struct",
-           "visual_attention_forward_train", "visual_attention_backward"]
+__all__ = ["moga_route", "moga_permute", "moga_group_attn", "stga_attn", "stga_attn_train", "stga_attn_mean",
+           "visual_attn_mean", "moga_balance_loss", "visual_attention_forward", "attn_workspace", "device_status",
+           "MogaError", "geom_struct", "visual_attention_forward_train", "visual_attention_backward"]
 
 
 def _ptr(t):
@@ -202,6 +202,25 @@ def stga_attn(q, k, v, geom: dict, softmax_scale: float | None = None, o_acc: to
                           ws.numel(), _stream()), "stga_attn")
     del keep
     return o_acc
+
+
+def stga_attn_train(q, k, v, geom: dict, softmax_scale: float | None = None, ws: torch.Tensor | None = None):
+    """Window-group and per-frame attention written to separate buffers, each with its
+    log2-domain log-sum-exp.  Returns (o_win, lse_win, o_frame, lse_frame)."""
+    N, H, hd = _check_qkv(q, k, v, device=False)
+    _check_geom(geom, N)
+    _on_device(q=q, k=k, v=v, ws=ws)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    o_win, o_frame = (torch.empty((N, H, hd), **f32) for _ in range(2))
+    lse_win, lse_frame = (torch.empty((N, H), **f32) for _ in range(2))
+    scale = 1.0 / math.sqrt(hd) if softmax_scale is None else softmax_scale
+    s, keep = geom_struct(geom)
+    ws = attn_workspace(q) if ws is None else ws
+    check(lib().stga_attn_train(_ptr(q), _ptr(k), _ptr(v), H, hd, ctypes.byref(s), scale, _ptr(o_win),
+                                _ptr(lse_win), _ptr(o_frame), _ptr(lse_frame), _ptr(ws), ws.numel(), _stream()),
+          "stga_attn_train")
+    del keep
+    return o_win, lse_win, o_frame, lse_frame
 
 
 def stga_attn_mean(q, k, v, geom: dict, o_acc: torch.Tensor, softmax_scale: float | None = None,

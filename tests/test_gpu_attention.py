@@ -1,10 +1,15 @@
-"""GPU parity: MoGA group attention, STGA window + frame attention and the layer output vs the fp64 oracle.
+"""GPU parity: MoGA group attention, the STGA window and frame branches (each on
+its own) and the layer output vs the fp64 oracle.
 
 Attention outputs from bf16 inputs must reach rel-L2 <= 1e-2 and max-abs
-<= 3e-2.  Small cases are compared element by element over every token and
-head; the 32k-token Wan-1.3B-shaped workload (the one the benchmark times) is
-compared on a stratified sample of tokens over every head, each sampled row
-computed by the oracle from its full definition.
+<= 3e-2, on every branch separately and on the output.  The branches come
+from the training forward, which writes each to its own buffer with the same
+kernels; the production call that adds both into the accumulator is checked
+to equal their fp32 sum bit for bit.  Small cases are compared element by
+element over every token and head; the 32k and 64k workloads are compared on
+a stratified sample of >= 4096 (token, head) rows over 8 heads covering every
+MoGA group, every window group, both sides of every shot cut and every frame,
+each sampled row computed by the oracle from its full definition.
 """
 import numpy as np
 import pytest
@@ -12,6 +17,7 @@ import pytest
 from _data import Case, assert_close
 from oracle import attention as oatt
 from oracle import layer as olayer
+from oracle import sample as osample
 from oracle import stga as ostga
 from synth import workloads as W
 
@@ -34,6 +40,8 @@ SMALL = {
 
 
 def _run_gpu(case, q_scale=1.0):
+    """Returns dict(moga, win, frame, static, out) as numpy fp32 and keeps the bf16 bit
+    patterns of the fused and the two-call layer output in _run_gpu.last_bits."""
     import torch
     import sparse_attention_long_moga_b200 as moga
     t = case.gpu()
@@ -44,16 +52,19 @@ def _run_gpu(case, q_scale=1.0):
     o_moga = moga.moga_group_attn(t["q"], t["k"], t["v"], perm, cu, gate, case.wl.M)
     o_moga_cpu = o_moga.cpu().numpy().copy()
     o_static = moga.stga_attn(t["q"], t["k"], t["v"], case.geom)          # zero-initialised accumulator
-    o_static_cpu = o_static.cpu().numpy()
+    o_win, _, o_frame, _ = moga.stga_attn_train(t["q"], t["k"], t["v"], case.geom)
+    # the accumulating call adds exactly the values the split call writes
+    assert torch.equal(o_static, (torch.zeros_like(o_win) + o_win) + o_frame), case.wl.name
     res = moga.visual_attention_forward(t["x"], t["w_r"], t["bias"], t["q"], t["k"], t["v"], case.wl.M,
                                         case.geom, case.wl.alpha)
     res_unfused = moga.visual_attention_forward(t["x"], t["w_r"], t["bias"], t["q"], t["k"], t["v"], case.wl.M,
                                                 case.geom, case.wl.alpha, fused_mean=False)
     moga.device_status()
-    out = res["out"].float().cpu().numpy()
     # bf16 bit patterns of the fused and the two-call output
-    _run_gpu.last_bits = (res["out"].view(torch.int16).cpu().numpy(), res_unfused["out"].view(torch.int16).cpu().numpy())
-    return o_moga_cpu, o_static_cpu, out
+    _run_gpu.last_bits = (res["out"].view(torch.int16).cpu().numpy(),
+                          res_unfused["out"].view(torch.int16).cpu().numpy())
+    return dict(moga=o_moga_cpu, win=o_win.cpu().numpy(), frame=o_frame.cpu().numpy(),
+                static=o_static.cpu().numpy(), out=res["out"].float().cpu().numpy())
 
 
 @pytest.fixture(scope="module", params=sorted(SMALL))
@@ -73,19 +84,29 @@ def small(request, cuda_device):
 
 
 def test_moga_attention_small(small):
-    case, ref, (o_moga, _, _), _ = small
-    assert_close(o_moga, ref["moga"], "moga " + case.wl.name)
+    case, ref, res, _ = small
+    assert_close(res["moga"], ref["moga"], "moga " + case.wl.name)
+
+
+def test_stga_window_small(small):
+    case, ref, res, _ = small
+    assert_close(res["win"], ref["win"], "window " + case.wl.name)
+
+
+def test_stga_frame_small(small):
+    case, ref, res, _ = small
+    assert_close(res["frame"], ref["frame"], "frame " + case.wl.name)
 
 
 def test_stga_attention_small(small):
-    case, ref, (_, o_static, _), _ = small
-    assert_close(o_static, ref["win"] + ref["frame"], "stga " + case.wl.name)
+    case, ref, res, _ = small
+    assert_close(res["static"], ref["win"] + ref["frame"], "stga " + case.wl.name)
 
 
 def test_layer_output_small(small):
-    case, ref, (_, _, out), _ = small
+    case, ref, res, _ = small
     # the output is bf16: add its half-ulp rounding to the budget through the same tolerance
-    assert_close(out, ref["out"], "layer " + case.wl.name)
+    assert_close(res["out"], ref["out"], "layer " + case.wl.name)
 
 
 def test_fused_mean_equals_two_calls(small):
@@ -102,58 +123,29 @@ def test_peaky_queries(cuda_device):
     q = q * 4.0
     g, p_g, _ = case.route64()
     scale = 1.0 / np.sqrt(case.wl.hd)
-    o_moga, o_static, _ = _run_gpu(case, q_scale=4.0)
-    assert_close(o_moga, oatt.moga(q, k, v, g, p_g, case.wl.M, scale), "peaky moga")
-    ref = oatt.grouped(q, k, v, ostga.window_groups(case.geom), scale) + \
-        oatt.grouped(q, k, v, ostga.frame_groups(case.geom), scale)
-    assert_close(o_static, ref, "peaky stga")
-
-
-def _sample_tokens(case, n_per_group=48, seed=0):
-    """Stratified token sample: every MoGA group, every frame of shot boundaries, every window."""
-    rs = np.random.default_rng(seed)
-    g, _, _ = case.route64()
-    toks = []
-    for i in range(case.wl.M):
-        mem = np.nonzero(g == i)[0]
-        if len(mem):
-            toks.append(rs.choice(mem, size=min(n_per_group, len(mem)), replace=False))
-            toks.append(mem[-1:])   # the ragged tail row of the group
-    hw = case.wl.hw
-    starts = np.concatenate([[0], np.cumsum(case.wl.shots)])
-    for f in sorted(set(int(s) for s in starts[:-1]) | set(int(s) - 1 for s in starts[1:])):
-        toks.append(f * hw + rs.integers(0, hw, 8))
-    return np.unique(np.concatenate(toks))
+    res = _run_gpu(case, q_scale=4.0)
+    assert_close(res["moga"], oatt.moga(q, k, v, g, p_g, case.wl.M, scale), "peaky moga")
+    assert_close(res["win"], oatt.grouped(q, k, v, ostga.window_groups(case.geom), scale), "peaky window")
+    assert_close(res["frame"], oatt.grouped(q, k, v, ostga.frame_groups(case.geom), scale), "peaky frame")
 
 
 @pytest.mark.parametrize("wl", [W.WAN13B_5S, W.MULTISHOT_10S], ids=lambda w: w.name)
 def test_sampled_rows_full_size(wl, cuda_device):
-    """Full-size workload in the benchmark's launch configuration; oracle on sampled rows."""
+    """Full-size workload in the benchmark's launch configuration; oracle on >= 4096
+    stratified (token, head) rows, every branch on its own."""
     case = Case(wl)
-    o_moga, o_static, out = _run_gpu(case)
+    res = _run_gpu(case)
     g, p_g, _ = case.route64()
-    toks = _sample_tokens(case)
+    rows = osample.stratified_rows(case.geom, g, wl.M, wl.H, n_heads=8, per_head=512)
+    assert sum(len(t) for t in rows.values()) >= 4096
     scale = 1.0 / np.sqrt(wl.hd)
-    wgroups = ostga.window_groups(case.geom)
-    owner = {}
-    for gi, (qt, _) in enumerate(wgroups):
-        for t in qt.tolist():
-            owner[t] = gi
-    ref_m = np.zeros((len(toks), wl.H, wl.hd))
-    ref_s = np.zeros_like(ref_m)
-    for h in range(wl.H):
+    got = {n: [] for n in ("moga", "win", "frame", "out")}
+    ref = {n: [] for n in got}
+    for h, toks in rows.items():
         qh, kh, vh = (case.head64(n, h) for n in ("q", "k", "v"))
-        for i in range(wl.M):
-            sel = np.nonzero(g[toks] == i)[0]
-            if len(sel) == 0:
-                continue
-            mem = np.nonzero(g == i)[0]
-            ref_m[sel, h] = oatt.rows_of_group(qh[toks[sel]], kh[mem], vh[mem], scale, p_g[toks[sel]])
-        for j, t in enumerate(toks.tolist()):
-            qt, kvt = wgroups[owner[t]]
-            fr = np.arange((t // wl.hw) * wl.hw, (t // wl.hw + 1) * wl.hw)
-            ref_s[j, h] = oatt.attend(qh[t:t + 1], kh[kvt], vh[kvt], scale)[0] + \
-                oatt.attend(qh[t:t + 1], kh[fr], vh[fr], scale)[0]
-    assert_close(o_moga[toks], ref_m, "moga sampled " + wl.name)
-    assert_close(o_static[toks], ref_s, "stga sampled " + wl.name)
-    assert_close(out[toks], (ref_m + ref_s) / 3.0, "layer sampled " + wl.name)
+        om, ow, of = osample.branch_rows(qh, kh, vh, toks, g, p_g, wl.M, case.geom, scale)
+        for n, r in (("moga", om), ("win", ow), ("frame", of), ("out", olayer.mean3(om, ow, of))):
+            ref[n].append(r)
+            got[n].append(res[n][toks, h])
+    for n in got:
+        assert_close(np.concatenate(got[n]), np.concatenate(ref[n]), "%s sampled %s" % (n, wl.name))

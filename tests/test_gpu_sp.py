@@ -4,8 +4,10 @@ The head pack / unpack kernels are pure data movement: bit-exact against the
 layout they are defined by (numpy reshape and transpose).  With one rank
 (an NCCL group of one GPU) the whole sequence-parallel forward must equal the
 single-GPU forward bit for bit (same kernels on the same data; the
-collectives are copies).  The multi-rank exchange is covered on CPU by
-tests/test_sp_cpu.py.
+collectives are copies), and, on the tiny workload, match the fp64 oracle's
+layer forward directly (routing and perm bit-exact, output within the
+attention tolerance, loss to 1e-5).  The multi-rank exchange is covered on
+CPU by tests/test_sp_cpu.py.
 """
 import datetime
 import socket
@@ -13,7 +15,8 @@ import socket
 import numpy as np
 import pytest
 
-from _data import Case
+from _data import LOSS_REL, Case, assert_close
+from oracle import layer as olayer
 from synth import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -73,3 +76,20 @@ def test_sp_one_rank_equals_single_gpu(name, nccl_world_of_one, cuda_device):
     assert torch.equal(got["out"], ref["out"])
     assert torch.equal(got["perm"], ref["perm"])
     assert float(got["loss"].item()) == float(ref["loss"].item())
+
+
+def test_sp_one_rank_against_oracle(nccl_world_of_one, cuda_device):
+    """The sequence-parallel forward checked against the oracle itself, not only
+    against the single-GPU CUDA path."""
+    import sparse_attention_long_moga_b200 as moga
+    from sparse_attention_long_moga_b200.sp import sp_visual_attention_forward
+    case = Case(W.TINY, with_qkv=True)
+    wl = case.wl
+    t = case.gpu(cuda_device)
+    got = sp_visual_attention_forward(t["x"], t["w_r"], t["bias"], t["q"], t["k"], t["v"], wl.M, case.geom, wl.alpha)
+    moga.device_status()
+    q, k, v = case.qkv64()
+    ref = olayer.forward(case.x64(), case.w64(), case.bias, q, k, v, wl.M, case.geom, wl.alpha)
+    assert np.array_equal(got["perm"].cpu().numpy(), ref["perm"].astype(np.int32))
+    assert_close(got["out"].float().cpu().numpy(), ref["out"], "sp layer output")
+    assert abs(float(got["loss"].item()) - ref["loss"]) <= LOSS_REL * abs(ref["loss"])
