@@ -27,6 +27,17 @@
  *     returns MOGA_ERR_CUDA.  Kernels never trap: a device-side wait that
  *     runs out of time records MOGA_ERR_TIMEOUT in a per-device error word,
  *     which moga_device_status() reports.
+ *   - Index arguments in device memory (group ids, perm, cu_seqlens) cannot
+ *     be checked on the host.  The permute records MOGA_ERR_BAD_INDEX for a
+ *     group id outside [0, M) in every build.  The checking build of this
+ *     library (libmoga_debug.so, compiled with -DMOGA_DEBUG; same ABI) also
+ *     checks, before each access, every perm entry against [0, N), that
+ *     cu_seqlens is a non-decreasing split inside [0, N], and that every
+ *     token row the kernels derive lies in [0, N); a failed check records
+ *     MOGA_ERR_BAD_INDEX and skips the access it guards (a bad cu_seqlens
+ *     skips the whole attention launch), so a bad index never reaches
+ *     memory.  In the default build such inputs are unchecked and their
+ *     result is undefined.
  *   - Limits: N * H < 2^31, 1 <= M <= 32, d % 8 == 0, hd in {64, 128}.
  */
 #ifndef MOGA_H
@@ -45,7 +56,8 @@ typedef enum {
   MOGA_ERR_UNSUPPORTED = 2,
   MOGA_ERR_WORKSPACE = 3,
   MOGA_ERR_CUDA = 4,
-  MOGA_ERR_TIMEOUT = 5
+  MOGA_ERR_TIMEOUT = 5,
+  MOGA_ERR_BAD_INDEX = 6
 } moga_status;
 
 typedef enum { MOGA_F32 = 0, MOGA_BF16 = 1 } moga_dtype;
@@ -95,9 +107,10 @@ moga_status moga_route(const void* x, const void* w_r, moga_dtype dt, const floa
  *   counts[i] = #{t : g_t = i}, cu_seqlens = exclusive prefix (cu[M] = N),
  *   perm[cu[i] + j] = the j-th smallest token index with g = i,
  *   *max_seqlen = max_i counts[i].
- * group_id: [N] int32, every value in [0, M) (values outside are not checked
- *           on the host; the kernels skip them and the result is then
- *           undefined)
+ * group_id: [N] int32, every value in [0, M); a value outside is skipped
+ *           (perm then holds fewer than N entries and counts sum to less
+ *           than N) and recorded as MOGA_ERR_BAD_INDEX in the device error
+ *           word, which moga_device_status() returns
  * perm [N], cu_seqlens [M+1], counts [M], max_seqlen [1]: int32 out
  * ws:       at least moga_permute_ws_bytes(N, M) bytes of scratch.
  */

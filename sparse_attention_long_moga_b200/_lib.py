@@ -13,9 +13,12 @@ import os
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libmoga.so")
+# the checking build (device-side index checks, same ABI); MOGA_DEBUG=1 in
+# the environment makes lib() load it instead of the default build
+DEBUG_LIB_PATH = os.path.join(PKG, "libmoga_debug.so")
 
 STATUS = {0: "MOGA_OK", 1: "MOGA_ERR_INVALID_ARG", 2: "MOGA_ERR_UNSUPPORTED", 3: "MOGA_ERR_WORKSPACE",
-          4: "MOGA_ERR_CUDA", 5: "MOGA_ERR_TIMEOUT"}
+          4: "MOGA_ERR_CUDA", 5: "MOGA_ERR_TIMEOUT", 6: "MOGA_ERR_BAD_INDEX"}
 MOGA_F32, MOGA_BF16 = 0, 1
 
 # exported symbol -> (restype, argtypes); the same list include/moga.h declares
@@ -74,10 +77,12 @@ class StgaGeom(ctypes.Structure):
                 ("aug_frames", _I32)]
 
 
-def load(path: str = LIB_PATH) -> ctypes.CDLL:
+def load(path: str | None = None) -> ctypes.CDLL:
+    if path is None:
+        path = DEBUG_LIB_PATH if os.environ.get("MOGA_DEBUG", "") not in ("", "0") else LIB_PATH
     if not os.path.exists(path):
-        raise ImportError("libmoga.so is not built (run sparse_attention_long_moga_b200.build); "
-                          "there is no fallback path")
+        raise ImportError("%s is not built (run sparse_attention_long_moga_b200.build); "
+                          "there is no fallback path" % os.path.basename(path))
     lib = ctypes.CDLL(path)
     for name, (res, args) in SIGNATURES.items():
         fn = getattr(lib, name)

@@ -13,6 +13,8 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmoga.so")
+# the checking build: device-side index checks (-DMOGA_DEBUG), same ABI
+DEBUG_LIB = os.path.join(PKG, "libmoga_debug.so")
 SOURCES = ["moga_lib.cu"]
 DEPS = ["tc_common.cuh", "route_tc.cu", "route_bwd.cu", "sp.cu", "qkv_route.cu", "attention_bwd.cu", "api_common.cu", "route.cu", "permute.cu", "permute_noalloc.cu", "mean_loss.cu", "attention.cu", "common.cuh"]
 
@@ -32,10 +34,10 @@ def flags(verbose: bool = False) -> list:
     return f
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     hdr = os.path.join(os.path.dirname(PKG), "include", "moga.h")
     srcs = [os.path.join(CSRC, s) for s in SOURCES + DEPS] + [hdr]
     return any(os.path.getmtime(s) > t for s in srcs if os.path.exists(s))
@@ -65,18 +67,25 @@ def check_register_split(ptxas_log: str) -> None:
         raise RuntimeError("could not find the attention kernel's register count in the ptxas report")
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not stale():
-        return LIB
-    tmp = LIB + ".tmp"
-    cmd = [nvcc()] + flags(True) + ["-o", tmp] + [os.path.join(CSRC, s) for s in SOURCES]
+def _compile(lib: str, extra: list, verbose: bool) -> None:
+    tmp = lib + ".tmp"
+    cmd = [nvcc()] + flags(True) + extra + ["-o", tmp] + [os.path.join(CSRC, s) for s in SOURCES]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if verbose or res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
     if res.returncode != 0:
         raise subprocess.CalledProcessError(res.returncode, cmd, res.stdout, res.stderr)
     check_register_split(res.stdout + res.stderr)
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+
+
+def build(force: bool = False, verbose: bool = False, debug: bool = True) -> str:
+    """Builds libmoga.so and (debug=True) the checking build libmoga_debug.so,
+    each only when a source is newer (or force); returns the default library."""
+    if force or stale(LIB):
+        _compile(LIB, [], verbose)
+    if debug and (force or stale(DEBUG_LIB)):
+        _compile(DEBUG_LIB, ["-DMOGA_DEBUG"], verbose)
     return LIB
 
 

@@ -27,7 +27,13 @@ moga_status check_launch(const char* what) {
 
 extern "C" const char* moga_last_error(void) { return moga::t_last_error; }
 
-extern "C" const char* moga_version(void) { return "moga-b200 0.1 (sm_100a)"; }
+extern "C" const char* moga_version(void) {
+#ifdef MOGA_DEBUG
+  return "moga-b200 0.2 (sm_100a, checking build: device-side index checks)";
+#else
+  return "moga-b200 0.2 (sm_100a)";
+#endif
+}
 
 extern "C" moga_status moga_device_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

@@ -138,10 +138,16 @@ __host__ __device__ __forceinline__ int window_token(const Params& p, int idx) {
   return frame * p.hw + row * p.w + col;
 }
 
+// Token (row of q, k, v and the outputs) at segment position idx.  The
+// checking build returns -1 for a row outside [0, N) (a bad perm entry) after
+// recording MOGA_ERR_BAD_INDEX; callers then skip the access.
 __device__ __forceinline__ int token_of(const Params& p, int idx) {
-  if (p.mode == MODE_MOGA) return __ldg(p.perm + idx);
-  if (p.mode == MODE_FRAME) return idx;
-  return window_token(p, idx);
+  const int t = p.mode == MODE_MOGA ? __ldg(p.perm + idx) : (p.mode == MODE_FRAME ? idx : window_token(p, idx));
+  if (kCheckIndices && (unsigned)t >= (unsigned)p.N) {
+    record_device_error(MOGA_ERR_BAD_INDEX);
+    return -1;
+  }
+  return t;
 }
 
 struct Tile {
@@ -160,6 +166,20 @@ struct GroupTable {
 // in the backward)
 __host__ __device__ void build_group_table(const Params& p, GroupTable& gt, int unit_rows = 2 * BM) {
   int size[32], order[32];
+  if (kCheckIndices) {
+    // cu_seqlens must split a range inside [0, N] without going backwards;
+    // otherwise the launch gets no tiles (every CTA builds the same table)
+    bool ok = load_ro(p.cu) >= 0 && load_ro(p.cu + p.M) <= p.N;
+    for (int i = 0; i < p.M; ++i) ok = ok && load_ro(p.cu + i) <= load_ro(p.cu + i + 1);
+    if (!ok) {
+#ifdef __CUDA_ARCH__
+      record_device_error(MOGA_ERR_BAD_INDEX);
+#endif
+      gt.n = 0;
+      gt.prefix[0] = 0;
+      return;
+    }
+  }
   for (int i = 0; i < p.M; ++i) {
     size[i] = load_ro(p.cu + i + 1) - load_ro(p.cu + i);
     order[i] = i;
@@ -252,6 +272,10 @@ gather3_kernel(const __grid_constant__ Params p, const uint4* __restrict__ q, co
   if (j >= p.N) return;
   const int lane = threadIdx.x & 31;
   const int src = MODE == MODE_MOGA ? __ldg(p.perm + j) : window_token(p, j);
+  if (kCheckIndices && (unsigned)src >= (unsigned)p.N) {
+    if (lane == 0) record_device_error(MOGA_ERR_BAD_INDEX);
+    return;
+  }
   const size_t so = (size_t)src * row_u4, dofs = (size_t)j * row_u4;
   for (int c = lane; c < row_u4; c += 32) {
     const uint4 a = __ldg(q + so + c);
@@ -511,8 +535,9 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
         // the fused mean reads this row of the accumulator in the epilogue:
         // start bringing it into L2 now, a whole work tile ahead
         const int q_pre = t.q_begin + qt * BM + row;
-        if (q_pre < t.q_end) {
-          const char* a = reinterpret_cast<const char*>(p.o_acc + ((size_t)token_of(p, q_pre) * p.H + t.head) * HD);
+        const int tok_pre = q_pre < t.q_end ? token_of(p, q_pre) : -1;
+        if (tok_pre >= 0) {
+          const char* a = reinterpret_cast<const char*>(p.o_acc + ((size_t)tok_pre * p.H + t.head) * HD);
 #pragma unroll
           for (int e = 0; e < HD * 4; e += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(a + e));
         }
@@ -601,8 +626,8 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
       tc_fence_before();
       mbar_arrive(bar(B_O_EMPTY + qt));   // O may be overwritten by the next tile now
       const int q_idx = t.q_begin + qt * BM + row;
-      if (q_idx < t.q_end) {
-        const int tok = token_of(p, q_idx);
+      const int tok = q_idx < t.q_end ? token_of(p, q_idx) : -1;
+      if (tok >= 0) {
         float scale = 1.0f / l_run;
         if (p.mode == MODE_MOGA) scale *= __ldg(p.gate + tok);
         float4* d4 = reinterpret_cast<float4*>(p.o_acc + ((size_t)tok * p.H + t.head) * HD);

@@ -141,6 +141,10 @@ bwd_prep_kernel(const __grid_constant__ BwdParams b, const uint4* __restrict__ q
   if (j >= p.N) return;
   const int lane = threadIdx.x & 31;
   const int src = MODE == MODE_MOGA ? __ldg(p.perm + j) : (MODE == MODE_WINDOW ? window_token(p, j) : j);
+  if (kCheckIndices && (unsigned)src >= (unsigned)p.N) {
+    if (lane == 0) record_device_error(MOGA_ERR_BAD_INDEX);
+    return;
+  }
   const int row_u4 = p.H * hd / 8;
   const size_t so = (size_t)src * row_u4, dofs = (size_t)j * row_u4;
   if (MODE != MODE_FRAME) {
@@ -539,7 +543,7 @@ bwd_dkdv_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUt
       tc_fence_after();
       const int kr = u.t_begin + row;
       const bool in = kr < u.t_end;
-      const int tok = in ? token_of(p, kr) : 0;
+      const int tok = in ? token_of(p, kr) : -1;
 #pragma unroll 1
       for (int part = 0; part < 2; ++part) {
         float g[HD];
@@ -549,7 +553,7 @@ bwd_dkdv_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUt
         if (part == 1)
 #pragma unroll
           for (int e = 0; e < HD; ++e) g[e] *= b.scale;   // dK = scale dS^T Q
-        if (in) add_rows<HD>(part == 0 ? b.dv : b.dk, tok, p.H, u.head, g);
+        if (tok >= 0) add_rows<HD>(part == 0 ? b.dv : b.dk, tok, p.H, u.head, g);
       }
     }
   }
@@ -695,7 +699,8 @@ bwd_dq_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUten
       tmem_wait_ld();
 #pragma unroll
       for (int e = 0; e < HD; ++e) g[e] *= b.scale;   // dQ = scale dS K
-      if (in) add_rows<HD>(b.dq, token_of(p, qr), p.H, u.head, g);
+      const int tok = in ? token_of(p, qr) : -1;
+      if (tok >= 0) add_rows<HD>(b.dq, tok, p.H, u.head, g);
     }
   }
   bwd_teardown<HD>(tmem);

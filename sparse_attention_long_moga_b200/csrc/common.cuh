@@ -25,6 +25,18 @@ __device__ __forceinline__ void record_device_error(int code) {
 
 __host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Index checks of the checking build (compiled with -DMOGA_DEBUG into
+// libmoga_debug.so): kernels test every index they take from a caller's
+// buffer (perm entries, cu_seqlens, token rows derived from them) before the
+// access it guards.  A failed check records MOGA_ERR_BAD_INDEX in the device
+// error word and skips that access (or, for a bad cu_seqlens, the whole
+// launch); nothing traps.  In the default build the checks compile away.
+#ifdef MOGA_DEBUG
+constexpr bool kCheckIndices = true;
+#else
+constexpr bool kCheckIndices = false;
+#endif
+
 // Limit of every bounded wait on an mbarrier, in SM clock cycles: about two
 // seconds at the maximum SM clock.  A wait that runs out records
 // MOGA_ERR_TIMEOUT in the device error word and the kernel returns.

@@ -38,7 +38,10 @@ tile_hist_kernel(const int32_t* __restrict__ g, int N, int M, int n_per, int K, 
     const int t = base + i * kThreads + threadIdx.x;
     if (t < N) {
       const int gi = __ldg(g + t);
-      if ((unsigned)gi < (unsigned)M) atomicAdd(&h[sort_key(gi, t, M, n_per)], 1);
+      if ((unsigned)gi < (unsigned)M)
+        atomicAdd(&h[sort_key(gi, t, M, n_per)], 1);
+      else
+        record_device_error(MOGA_ERR_BAD_INDEX);   // skipped here and by the scatter
     }
   }
   __syncthreads();

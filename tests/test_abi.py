@@ -119,6 +119,27 @@ def test_mean_and_loss_argument_checks(lib):
 
 def test_version(lib):
     assert b"sm_100a" in lib.moga_version()
+    assert b"checking" not in lib.moga_version()
+
+
+def test_status_codes_match_header():
+    text = open(HEADER).read()
+    enum = dict((n, int(v)) for n, v in re.findall(r"(MOGA_OK|MOGA_ERR_\w+)\s*=\s*(\d+)", text))
+    assert {v: k for k, v in enum.items()} == _lib.STATUS
+
+
+def test_checking_build_loads_and_validates_like_the_default():
+    """The checking build (device-side index checks) exports the same ABI and
+    rejects the same host-side arguments; its kernels need a GPU."""
+    build()
+    dbg = _lib.load(_lib.DEBUG_LIB_PATH)
+    assert b"checking build" in dbg.moga_version()
+    for name in declared_functions():
+        assert hasattr(dbg, name), name
+    # host validation is shared code: a bad M is refused before any launch
+    assert dbg.moga_permute(ctypes.c_void_p(16), 100, 33, ctypes.c_void_p(16), ctypes.c_void_p(16),
+                            ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16), 1 << 20, None) == 1
+    assert b"M=33" in dbg.moga_last_error()
 
 
 def test_batch_sp_and_projection_workspace_sizes(lib):
