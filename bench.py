@@ -44,11 +44,11 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # DRAM bytes (read + write) of one moga_group_attn call on the 5 s Wan-1.3B
-# workload (32,760 tokens x 12 heads x 128), from an ncu --set full capture:
-# gather3_kernel<0> 302.1 + 263.1 MB, attn_kernel<128> (MoGA launch)
-# 305.1 + 162.2 MB.  Set to None whenever either kernel changes, until it is
-# captured again.
-CALL_TRAFFIC_BYTES = 1.0325e9
+# workload (32,760 tokens x 12 heads x 128), from an ncu capture of the
+# current kernels: gather3_kernel<0> 302.06 + 259.95 MB, attn_kernel<128>
+# (MoGA launch) 304.74 + 158.97 MB.  Set to None whenever either kernel
+# changes, until it is captured again.
+CALL_TRAFFIC_BYTES = 1.0257e9
 CALL_TRAFFIC_UNITS = 32760 * 12 * 128
 CALL_TRAFFIC_SOURCE = "ncu dram__bytes_read.sum + dram__bytes_write.sum, gather3_kernel<0> + attn_kernel<128> MoGA launch"
 
@@ -345,6 +345,87 @@ def router_kind(wl):
 
 # ----------------------------------------------------------------------------- GPU arm
 
+def run_e2e(args, world, dev, inp, step, out, loss, flush, stream, N):
+    """The step end to end through the C ABI: every step copies its inputs in
+    from pinned host memory and its result out, inside the timed region."""
+    import torch
+    import torch.distributed as dist
+    import sparse_attention_long_moga_b200 as moga
+    hx, hq, hk, hv = (torch.from_numpy(inp[n].view(np.int16)).pin_memory() for n in ("x", "q", "k", "v"))
+    hosts = (hx, hq, hk, hv)
+    hout = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    hloss = torch.empty(1, dtype=torch.float64).pin_memory()
+    h2d = sum(a.numel() * a.element_size() for a in hosts)
+    d2h = hout.numel() * 2 + 8
+    bf = lambda t: t.view(torch.bfloat16)  # noqa: E731
+    # (a) serial: each step copies its inputs in, runs, and copies its result
+    # out on one stream
+    xd, qd, kd, vd = (torch.empty_like(a, device=dev) for a in hosts)
+    e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        e_evs[i][0].record(stream)
+        for dst, src in zip((xd, qd, kd, vd), hosts):
+            dst.copy_(src, non_blocking=True)
+        step(bf(xd), bf(qd), bf(kd), bf(vd))
+        hout.copy_(out, non_blocking=True)
+        hloss.copy_(loss, non_blocking=True)
+        e_evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    serial_ms = sum(a.elapsed_time(b) for a, b in e_evs)
+    want_out, want_loss = hout.clone(), hloss.clone()
+    # (b) pipelined, as a stream of requests is served: step i's inputs go
+    # into buffer set i % 2 on a host-to-device stream and its result leaves
+    # output buffer i % 2 on a device-to-host stream, so the copies of one
+    # step overlap the kernels of its neighbours.  Every step's copies lie
+    # inside the timed region; its 400 MB of fresh inputs exceed L2.
+    ins = [(xd, qd, kd, vd), tuple(torch.empty_like(a, device=dev) for a in hosts)]
+    outs = [(out, loss), (torch.empty_like(out), torch.empty_like(loss))]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: [torch.cuda.Event() for _ in range(args.steps)]  # noqa: E731
+    copied, computed, returned = ev(), ev(), ev()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    s_in.wait_stream(stream)
+    for i in range(args.steps):
+        b = i & 1
+        if i >= 2:
+            s_in.wait_event(computed[i - 2])      # step i-2 has read buffer set b
+        with torch.cuda.stream(s_in):
+            for dst, src in zip(ins[b], hosts):
+                dst.copy_(src, non_blocking=True)
+        copied[i].record(s_in)
+        stream.wait_event(copied[i])
+        if i >= 2:
+            stream.wait_event(returned[i - 2])    # output buffer b has left
+        step(*(bf(t) for t in ins[b]), out=outs[b][0], loss=outs[b][1])
+        computed[i].record(stream)
+        s_out.wait_event(computed[i])
+        with torch.cuda.stream(s_out):
+            hout.copy_(outs[b][0], non_blocking=True)
+            hloss.copy_(outs[b][1], non_blocking=True)
+        returned[i].record(s_out)
+    stream.wait_event(returned[-1])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    pipe_ms = t0.elapsed_time(t1)
+    moga.device_status()
+    # the last step's result crossed the streams intact
+    if not (torch.equal(hout, want_out) and torch.equal(hloss, want_loss)):
+        raise RuntimeError("pipelined end-to-end result differs from the serial one")
+    e2e_value = job_throughput(world, N, args.steps, max_over_ranks(pipe_ms, dev))
+    e2e_serial = job_throughput(world, N, args.steps, max_over_ranks(serial_ms, dev))
+    return {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "pipelined": True, "ms_per_step": pipe_ms / args.steps, "serial_value": e2e_serial,
+            "serial_ms_per_step": serial_ms / args.steps}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -465,76 +546,9 @@ def run_ours(args):
     value = job_throughput(world, N, args.steps, job_ms)
 
     # ---- end to end through the C ABI: pinned host inputs in, result out
-    hx, hq, hk, hv = (torch.from_numpy(inp[n].view(np.int16)).pin_memory() for n in ("x", "q", "k", "v"))
-    hosts = (hx, hq, hk, hv)
-    hout = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
-    hloss = torch.empty(1, dtype=torch.float64).pin_memory()
-    h2d = sum(a.numel() * a.element_size() for a in hosts)
-    d2h = hout.numel() * 2 + 8
-    bf = lambda t: t.view(torch.bfloat16)  # noqa: E731
-    # (a) serial: each step copies its inputs in, runs, and copies its result
-    # out on one stream
-    xd, qd, kd, vd = (torch.empty_like(a, device=dev) for a in hosts)
-    e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush.zero_()
-        e_evs[i][0].record(stream)
-        for dst, src in zip((xd, qd, kd, vd), hosts):
-            dst.copy_(src, non_blocking=True)
-        step(bf(xd), bf(qd), bf(kd), bf(vd))
-        hout.copy_(out, non_blocking=True)
-        hloss.copy_(loss, non_blocking=True)
-        e_evs[i][1].record(stream)
-    torch.cuda.synchronize()
-    serial_ms = sum(a.elapsed_time(b) for a, b in e_evs)
-    want_out, want_loss = hout.clone(), hloss.clone()
-    # (b) pipelined, as a stream of requests is served: step i's inputs go
-    # into buffer set i % 2 on a host-to-device stream and its result leaves
-    # output buffer i % 2 on a device-to-host stream, so the copies of one
-    # step overlap the kernels of its neighbours.  Every step's copies lie
-    # inside the timed region; its 400 MB of fresh inputs exceed L2.
-    ins = [(xd, qd, kd, vd), tuple(torch.empty_like(a, device=dev) for a in hosts)]
-    outs = [(out, loss), (torch.empty_like(out), torch.empty_like(loss))]
-    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev = lambda: [torch.cuda.Event() for _ in range(args.steps)]  # noqa: E731
-    copied, computed, returned = ev(), ev(), ev()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t0.record(stream)
-    s_in.wait_stream(stream)
-    for i in range(args.steps):
-        b = i & 1
-        if i >= 2:
-            s_in.wait_event(computed[i - 2])      # step i-2 has read buffer set b
-        with torch.cuda.stream(s_in):
-            for dst, src in zip(ins[b], hosts):
-                dst.copy_(src, non_blocking=True)
-        copied[i].record(s_in)
-        stream.wait_event(copied[i])
-        if i >= 2:
-            stream.wait_event(returned[i - 2])    # output buffer b has left
-        step(*(bf(t) for t in ins[b]), out=outs[b][0], loss=outs[b][1])
-        computed[i].record(stream)
-        s_out.wait_event(computed[i])
-        with torch.cuda.stream(s_out):
-            hout.copy_(outs[b][0], non_blocking=True)
-            hloss.copy_(outs[b][1], non_blocking=True)
-        returned[i].record(s_out)
-    stream.wait_event(returned[-1])
-    t1.record(stream)
-    torch.cuda.synchronize()
-    pipe_ms = t0.elapsed_time(t1)
-    moga.device_status()
-    # the last step's result crossed the streams intact
-    if not (torch.equal(hout, want_out) and torch.equal(hloss, want_loss)):
-        raise RuntimeError("pipelined end-to-end result differs from the serial one")
-    e2e_value = job_throughput(world, N, args.steps, max_over_ranks(pipe_ms, dev))
-    e2e_serial = job_throughput(world, N, args.steps, max_over_ranks(serial_ms, dev))
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, world, dev, inp, step, out, loss, flush, stream, N)
 
     counts_h = counts.cpu().numpy()
     fl_moga = moga_flops(counts_h, H, hd)
@@ -567,9 +581,7 @@ def run_ours(args):
             counts_h.astype(np.float64) ** 2))},
         "mean_fused_into_stga": bool(args.fused_mean),
         "route_permute_hbm": route_permute_hbm(wl, call_ms, pk),
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "pipelined": True, "ms_per_step": pipe_ms / args.steps, "serial_value": e2e_serial,
-                "serial_ms_per_step": serial_ms / args.steps},
+        "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
@@ -962,6 +974,8 @@ def main():
                     help="suite workload (default: %s for the forward, %s for the other modes)"
                     % (HEADLINE.name, SECONDARY.name))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end leg (host copies), e.g. for a profiler's launch list")
     ap.add_argument("--fused-mean", action="store_true",
                     help="run stga_attn_mean (mean inside the STGA frame pass) instead of stga_attn + visual_attn_mean")
     ap.add_argument("--train", action="store_true",

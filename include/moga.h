@@ -134,6 +134,9 @@ moga_status moga_permute(const int32_t* group_id, int64_t N, int32_t M,
  *     Nothing in it needs to start at zero; each call writes what it reads.
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
+ *     The address is kept for the life of the process: it does not survive
+ *     cudaDeviceReset() or another teardown of the device's primary context,
+ *     after which this call must not be used in the same process.
  *   - Allocates nothing and calls no allocating routine. */
 moga_status moga_permute_noalloc(const int32_t* group_id, int64_t N, int32_t M,
                                  int32_t* perm, int32_t* cu_seqlens, int32_t* counts,

@@ -24,7 +24,10 @@
 //     threads) race on the array: serialise them.
 //   * The first call on a device looks up the array's device address with
 //     cudaGetSymbolAddress (with that device current) and caches it; make
-//     that first call before any stream capture.
+//     that first call before any stream capture.  The cache lives as long as
+//     the process and is never refreshed: after cudaDeviceReset() (or any
+//     other teardown of the primary context) the cached address is stale, so
+//     the entry point must not be called again in that process.
 #include <mutex>
 
 #include "common.cuh"

@@ -14,8 +14,10 @@
 //              the slot's NP partial logits into fp32 registers (round to
 //              nearest), then after the last slice adds the bias and takes
 //              softmax, argmax, gate and the fixed-order per-warp sum of p(i|x)
-//   warp 4     producer: TMA loads of x tiles (up to 4 chunks of 32 tokens
-//              x 64 k, 128B swizzle) and of the matching W_r^T tile (NP
+//   warp 4     producer: TMA loads of x tiles (four chunks of 32 tokens x
+//              64 k as one 128-row box, or the chunks one by one for a
+//              CTA's last, partial group; 128B swizzle, the same shared-
+//              memory layout either way) and of the matching W_r^T tile (NP
 //              groups x 64 k) into a ring of 11-12 stages (~220 KB of
 //              shared memory, enough bytes in flight per SM to cover the
 //              HBM latency at the per-SM share of the bandwidth)
@@ -105,7 +107,7 @@ __device__ __forceinline__ void ld_slot(uint32_t taddr, float* v) {
 template <int NP>
 __global__ void __launch_bounds__(kThreads, 1)
 route_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tm_x,
-                const __grid_constant__ CUtensorMap tm_w) {
+                const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x4) {
   using C = Cfg<NP>;
   constexpr int kStages = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -149,6 +151,7 @@ route_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_x)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_w)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_x4)) : "memory");
       int c = 0;
       int last[kStages];
       for (int s = 0; s < kStages; ++s) last[s] = -1;
@@ -161,8 +164,11 @@ route_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtens
           if (!(ok = mbar_wait(bar(B_EMPTY + st), ph ^ 1, abort_flag, timeout))) break;
           mbar_arrive_expect_tx(bar(B_FULL + st), nch * kChunkBytes + C::kWBytes);
           const uint32_t dst = sbase + st * C::kStageBytes;
-          for (int j = 0; j < nch; ++j)
-            tma_load_2d(dst + j * kChunkBytes, &tm_x, kt * BK, (c0 + j) * kChunk, bar(B_FULL + st));
+          if (nch == 4)   // the four chunks as one 128-row box
+            tma_load_2d(dst, &tm_x4, kt * BK, c0 * kChunk, bar(B_FULL + st));
+          else
+            for (int j = 0; j < nch; ++j)
+              tma_load_2d(dst + j * kChunkBytes, &tm_x, kt * BK, (c0 + j) * kChunk, bar(B_FULL + st));
           tma_load_2d(dst + kXBytes, &tm_w, kt * BK, 0, bar(B_FULL + st));
           last[st] = c;
         }
@@ -326,15 +332,16 @@ static int sm_count() {
 template <int NP>
 static moga_status launch_np(const Params& prm, const void* wt, int dpad, const void* x, cudaStream_t s) {
   using C = Cfg<NP>;
-  CUtensorMap mx, mw;
+  CUtensorMap mx, mw, mx4;
   moga_status st;
   if ((st = make_map(&mx, x, prm.N, prm.d, (int64_t)prm.d * 2, kChunk)) != MOGA_OK) return st;
+  if ((st = make_map(&mx4, x, prm.N, prm.d, (int64_t)prm.d * 2, BT)) != MOGA_OK) return st;
   if ((st = make_map(&mw, wt, NP, dpad, (int64_t)dpad * 2, NP)) != MOGA_OK) return st;
   cudaError_t e = cudaFuncSetAttribute(route_tc_kernel<NP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return fail(MOGA_ERR_CUDA, "moga_route: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
   const int grid = std::min(prm.n_chunks, sm_count());
-  route_tc_kernel<NP><<<grid, kThreads, C::kSmemBytes, s>>>(prm, mx, mw);
+  route_tc_kernel<NP><<<grid, kThreads, C::kSmemBytes, s>>>(prm, mx, mw, mx4);
   return check_launch("moga_route");
 }
 

@@ -25,7 +25,9 @@ def _outputs(torch, dev, N, M):
             torch.empty(M, dtype=torch.int32, device=dev), torch.empty(1, dtype=torch.int32, device=dev))
 
 
-@pytest.mark.parametrize("N,M", [(282360, 20), (32760, 5)])
+# the last two cases reach the array's bound: 2048 tiles of 2048 tokens at
+# 32 groups fill both the histogram and the offset halves of the scratch
+@pytest.mark.parametrize("N,M", [(282360, 20), (32760, 5), (4194304, 32), (4194304 - 77, 32)])
 def test_noalloc_matches_workspace_permute_twice(cuda_device, N, M):
     import torch
     import sparse_attention_long_moga_b200 as moga
