@@ -51,3 +51,20 @@ def test_moga_flops_equal_dense_mask(N, M):
     counts = opermute.permute(g, M)[2]
     pairs = int(np.count_nonzero(g[:, None] == g[None, :]))
     assert bench.moga_flops(counts, 3, 64) == 4.0 * 3 * 64 * pairs
+
+
+@pytest.mark.parametrize("wl", CASES, ids=lambda w: w.name)
+def test_cpu_baseline_row_costs_match_flop_count(wl):
+    """The CPU baseline scales its sampled attention rows to the whole layer by
+    the keys each (token, head) row attends over in the three branches; summed
+    over all rows (times 4 hd) that must be exactly the benchmark's FLOP count
+    of the three branches."""
+    rs = np.random.default_rng(5)
+    g = rs.integers(0, wl.M, wl.N)
+    counts = np.bincount(g, minlength=wl.M)
+    kv_win = np.zeros(wl.N, dtype=np.int64)
+    for qt, kvt in ostga.window_groups(W.stga_shape(wl)):
+        kv_win[qt] = len(kvt)
+    cost_tok = counts[g] + kv_win + wl.hw
+    flops_from_rows = 4.0 * wl.hd * float(cost_tok.sum()) * wl.H
+    assert flops_from_rows == bench.moga_flops(counts, wl.H, wl.hd) + bench.stga_flops(wl)
