@@ -204,18 +204,34 @@ def _f64(a):
     return W.bf16_bits_to_f64(a) if a.dtype == np.uint16 else a.astype(np.float64)
 
 
-def oracle_sample(wl, inputs, seed=1, n_heads=8, per_head=512):
+def oracle_route_all(wl, inputs):
+    """The oracle's routing of all N tokens (row chunks of ROUTE_CHUNK, one after another)."""
+    from oracle import route as oroute
+    N = wl.N
+    w = _f64(inputs["w_r"])
+    g = np.empty(N, dtype=np.int64)
+    p_g = np.empty(N)
+    p = np.empty((N, wl.M))
+    for a in range(0, N, ROUTE_CHUNK):
+        b = min(a + ROUTE_CHUNK, N)
+        g[a:b], p_g[a:b], p[a:b] = oroute.route(_f64(inputs["x"][a:b]), w, W.bias_f64(wl))
+    return g, p_g, p
+
+
+def oracle_sample(wl, inputs, seed=1, n_heads=8, per_head=512, routed=None, route_fraction=1.0):
     """Times the fp64 oracle as it stands on a bounded sample of one layer forward.
 
-    Route over all N tokens (in row chunks of ROUTE_CHUNK, one after another),
-    permute and loss over all N; then, for n_heads heads spread over [0, H),
-    the three attention branches and the mean at a stratified sample of
-    per_head tokens (every MoGA group, window group, both sides of every cut
-    and every frame), each row computed from its full definition.  The
-    attention time is extrapolated to the whole layer by the exact per-row
-    cost (keys per row over the three branches, summed over all tokens and
-    heads); the per-head widening of q, k, v to float64 is timed apart and
-    scaled by heads.  Returns (tokens/s, details)."""
+    Route over all N tokens (or, with route_fraction < 1, over a contiguous
+    share of them, scaled to N by token count; `routed` then supplies the
+    routing of all tokens, computed outside the timed part), permute and loss
+    over all N; then, for n_heads heads spread over [0, H), the three attention
+    branches and the mean at a stratified sample of per_head tokens (every
+    MoGA group, window group, both sides of every cut and every frame), each
+    row computed from its full definition.  The attention time is
+    extrapolated to the whole layer by the exact per-row cost (keys per row
+    over the three branches, summed over all tokens and heads); the per-head
+    widening of q, k, v to float64 is timed apart and scaled by heads.
+    Returns (tokens/s, details)."""
     from oracle import layer as olayer
     from oracle import permute as opermute
     from oracle import route as oroute
@@ -223,17 +239,21 @@ def oracle_sample(wl, inputs, seed=1, n_heads=8, per_head=512):
     from oracle import stga as ostga
 
     N, H = wl.N, wl.H
-    w = _f64(inputs["w_r"])
+    if route_fraction >= 1.0 or routed is None:
+        t0 = time.perf_counter()
+        g, p_g, p = oracle_route_all(wl, inputs)
+        t_route = time.perf_counter() - t0
+    else:
+        g, p_g, p = routed
+        n_r = max(1, int(N * route_fraction))
+        a = (seed * 7919 * ROUTE_CHUNK) % max(N - n_r, 1)
+        t0 = time.perf_counter()
+        oroute.route(_f64(inputs["x"][a:a + n_r]), _f64(inputs["w_r"]), W.bias_f64(wl))
+        t_route = (time.perf_counter() - t0) * N / n_r
     t0 = time.perf_counter()
-    g = np.empty(N, dtype=np.int64)
-    p_g = np.empty(N)
-    p = np.empty((N, wl.M))
-    for a in range(0, N, ROUTE_CHUNK):
-        b = min(a + ROUTE_CHUNK, N)
-        g[a:b], p_g[a:b], p[a:b] = oroute.route(_f64(inputs["x"][a:b]), w, W.bias_f64(wl))
     perm, cu, counts, _ = opermute.permute(g, wl.M)
     olayer.balance_loss(counts, p, wl.alpha)
-    t_route = time.perf_counter() - t0
+    t_route += time.perf_counter() - t0
 
     geom = W.stga_shape(wl)
     scale = 1.0 / math.sqrt(wl.hd)
@@ -264,16 +284,21 @@ def oracle_sample(wl, inputs, seed=1, n_heads=8, per_head=512):
     t_mean_all = t_mean * (N * H) / n_rows
     t_layer = t_route + t_attn + t_mean_all
     return N / t_layer, dict(t_route_s=t_route, t_conv_s=t_conv, t_rows_s=t_rows, t_mean_s=t_mean,
-                             heads=len(rows), rows=n_rows, t_layer_extrapolated_s=t_layer)
+                             heads=len(rows), rows=n_rows, t_layer_extrapolated_s=t_layer,
+                             route_fraction=min(route_fraction, 1.0) if routed is not None else 1.0)
 
 
 def oracle_sample_text(wl, det):
-    return ("fp64 oracle, extrapolated: route+permute+loss over all %d tokens (%.1f s); attention (MoGA, window, "
-            "frame) + mean at a stratified sample of %d (token, head) rows over %d of %d heads covering every "
-            "group, window group, cut side and frame (%.1f s rows + %.1f s widening), scaled by exact per-row "
-            "key counts to all %d x %d rows -> %.0f s per layer"
-            % (wl.N, det["t_route_s"], det["rows"], det["heads"], wl.H, det["t_rows_s"], det["t_conv_s"], wl.N,
-               wl.H, det["t_layer_extrapolated_s"]))
+    if det.get("route_fraction", 1.0) < 1.0:
+        route = ("route timed on a contiguous %.1f %% of the tokens and scaled to all %d, permute+loss over all "
+                 "(%.1f s)" % (100 * det["route_fraction"], wl.N, det["t_route_s"]))
+    else:
+        route = "route+permute+loss over all %d tokens (%.1f s)" % (wl.N, det["t_route_s"])
+    return ("fp64 oracle, extrapolated: %s; attention (MoGA, window, frame) + mean at a stratified sample of %d "
+            "(token, head) rows over %d of %d heads covering every group, window group, cut side and frame "
+            "(%.1f s rows + %.1f s widening), scaled by exact per-row key counts to all %d x %d rows -> %.0f s "
+            "per layer" % (route, det["rows"], det["heads"], wl.H, det["t_rows_s"], det["t_conv_s"], wl.N, wl.H,
+                           det["t_layer_extrapolated_s"]))
 
 
 def host_cores():
@@ -309,11 +334,17 @@ def run_reference(args):
         return 0
     wl = pick_workload(args, HEADLINE)
     inputs = make_inputs(wl)
+    # the routing of all tokens once, outside the steps: it defines the groups
+    # the attention sample needs; each step times the router on an eighth of
+    # the tokens and 4 heads of attention rows, so a run of tens of steps ends
+    # within a few minutes on a few host cores
+    routed = oracle_route_all(wl, inputs)
+    frac = 1.0 if wl.N <= 65536 else 0.125
     for i in range(args.warmup):
-        oracle_sample(wl, inputs, seed=100 + i, n_heads=2, per_head=256)
+        oracle_sample(wl, inputs, seed=100 + i, n_heads=2, per_head=256, routed=routed, route_fraction=frac)
     t0 = time.perf_counter()
-    # 4 heads per step keeps a 10-step run within a few minutes on a few host cores
-    res = [oracle_sample(wl, inputs, seed=1 + s, n_heads=4) for s in range(args.steps)]
+    res = [oracle_sample(wl, inputs, seed=1 + s, n_heads=4, routed=routed, route_fraction=frac)
+           for s in range(args.steps)]
     el = time.perf_counter() - t0
     value = float(statistics.median([r[0] for r in res]))
     det = res[len(res) // 2][1]
@@ -593,6 +624,75 @@ def run_ours(args):
     if world > 1:
         dist.destroy_process_group()
     del keep
+    return 0
+
+
+def run_route(args):
+    """The router alone on the workload's x and W_r (and the permute of its
+    group ids): CUDA-event time per call with L2 flushed in between, GB/s and
+    fraction of the measured HBM bandwidth.  Prints one JSON line (not the
+    forward headline line)."""
+    import torch
+    import sparse_attention_long_moga_b200 as moga
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    wl = pick_workload(args, HEADLINE)
+    redraw = W.redraw_map(wl)
+    x_st = W.x_stored(wl, redraw)
+    if x_st.dtype != np.uint16:
+        raise SystemExit("--route times the bf16 router; %s has fp32 input" % wl.name)
+    x = torch.from_numpy(x_st.view(np.int16)).to(dev).view(torch.bfloat16)
+    w = torch.from_numpy(W.w_r_stored(wl).view(np.int16)).to(dev).view(torch.bfloat16)
+    bias = None
+    if wl.bias0 is not None:
+        bias = torch.from_numpy(W.bias_f64(wl).astype(np.float32)).to(dev)
+    del x_st
+    N, d, M = wl.N, wl.d, wl.M
+    L = moga._lib.lib()
+    P = moga._ptr
+    sp = moga._stream()
+    stream = torch.cuda.current_stream()
+    g = torch.empty(N, dtype=torch.int32, device=dev)
+    gate = torch.empty(N, dtype=torch.float32, device=dev)
+    rws = torch.empty(max(L.moga_route_ws_bytes(N, d, M), 16), dtype=torch.uint8, device=dev)
+    pws = torch.empty(max(L.moga_permute_ws_bytes(N, M), 16), dtype=torch.uint8, device=dev)
+    perm = torch.empty(N, dtype=torch.int32, device=dev)
+    cu = torch.empty(M + 1, dtype=torch.int32, device=dev)
+    counts = torch.empty(M, dtype=torch.int32, device=dev)
+    mx = torch.empty(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def route():
+        moga.check(L.moga_route(P(x), P(w), moga.MOGA_BF16, P(bias) if bias is not None else None, N, d, M, P(g),
+                                P(gate), P(rws), rws.numel(), sp), "route")
+
+    def permute():
+        moga.check(L.moga_permute(P(g), N, M, P(perm), P(cu), P(counts), P(mx), P(pws), pws.numel(), sp), "permute")
+
+    for _ in range(args.warmup):
+        route()
+        permute()
+    moga.device_status()
+    ms = {"route": [], "permute": []}
+    for _ in range(args.steps):
+        for name, fn in (("route", route), ("permute", permute)):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            ms[name].append(a.elapsed_time(b))
+    moga.device_status()
+    pk, pk_kind = peaks()
+    hbm = route_permute_hbm(wl, ms, pk)
+    line = {"metric": "router and permute alone, GB/s (bf16 x)", "value": hbm["unit"]["gbs"], "unit": "GB/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "dtype": "bf16", "data": "synthetic (seeded counter-based generator; no dataset)",
+            "config": {"workload": wl.name, "tokens": N, "d": d, "M": M,
+                       "l2": "flushed before every timed call (256 MiB write)"},
+            "route_permute_hbm": hbm, "peak_kind": "%s HBM copy bandwidth" % pk_kind}
+    print(json.dumps(line), flush=True)
     return 0
 
 
@@ -980,6 +1080,8 @@ def main():
                     help="run stga_attn_mean (mean inside the STGA frame pass) instead of stga_attn + visual_attn_mean")
     ap.add_argument("--train", action="store_true",
                     help="time the training step (saving forward + backward) instead of the forward")
+    ap.add_argument("--route", action="store_true",
+                    help="time the router and the permute alone (L2 flushed before each call)")
     ap.add_argument("--qkv", action="store_true",
                     help="time the router fused into the Q/K/V projection against GEMM + route")
     ap.add_argument("--sp", action="store_true",
@@ -997,6 +1099,8 @@ def main():
         return run_sp(args)
     if args.qkv:
         return run_qkv(args)
+    if args.route:
+        return run_route(args)
     return run_ours(args)
 
 
