@@ -501,11 +501,14 @@ def run_ours(args):
     o_acc = torch.empty((N, H, hd), dtype=torch.float32, device=dev)
     out = torch.empty((N, H, hd), dtype=torch.bfloat16, device=dev)
     loss = torch.empty(1, dtype=torch.float64, device=dev)
-    aws = torch.empty(L.moga_attn_ws_bytes(N, H, hd), dtype=torch.uint8, device=dev)
+    ws_fn = L.visual_attn_ws_bytes if args.combined else L.moga_attn_ws_bytes
+    aws = torch.empty(ws_fn(N, H, hd), dtype=torch.uint8, device=dev)
     gs, keep = moga.geom_struct(geom)
     scale = 1.0 / math.sqrt(hd)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    if not args.fused_mean:
+    if args.combined:
+        CALLS = ("route", "permute", "visual_attn_branches", "visual_attn_mean", "moga_balance_loss")
+    elif not args.fused_mean:
         CALLS = ("route", "permute", "moga_group_attn", "stga_attn", "visual_attn_mean", "moga_balance_loss")
     else:
         CALLS = ("route", "permute", "moga_group_attn", "stga_attn_mean", "moga_balance_loss")
@@ -523,6 +526,16 @@ def run_ours(args):
         mark(1)
         c(L.moga_permute(P(g), N, M, P(perm), P(cu), P(counts), P(mx), P(pws), pws.numel(), sp), "permute")
         mark(2)
+        if args.combined:
+            # the three branches with one gather of Q, K, V into both orders
+            c(L.visual_attn_branches(P(qd), P(kd), P(vd), N, H, hd, P(perm), P(cu), M, P(gate),
+                                     moga.ctypes.byref(gs), scale, P(o_acc), P(aws), aws.numel(), sp), "branches")
+            mark(3)
+            c(L.visual_attn_mean(P(o_acc), o_acc.numel(), P(out), sp), "mean")
+            mark(len(CALLS) - 1)
+            c(L.moga_balance_loss(P(counts), P(rws), N, M, wl.alpha, P(loss), sp), "loss")
+            mark(len(CALLS))
+            return
         c(L.moga_group_attn(P(qd), P(kd), P(vd), N, H, hd, P(perm), P(cu), M, P(gate), scale, P(o_acc), P(aws),
                             aws.numel(), sp), "moga")
         mark(3)
@@ -542,6 +555,8 @@ def run_ours(args):
     # route 2 (W_r^T copy + tensor-core router), permute 3, MoGA gather + attention 2,
     # STGA gather + window + frame 3, loss 1 (+ mean 1 and its tail when not fused)
     launches_per_step = 2 + 3 + 2 + 3 + 1
+    if args.combined:   # one gather instead of two
+        launches_per_step -= 1
     if not args.fused_mean:
         launches_per_step += 1 + (1 if (N * H * hd) % 8 else 0)
 
@@ -566,7 +581,7 @@ def run_ours(args):
         evl[-1].synchronize()
         for j, name in enumerate(CALLS):
             call_ms[name].append(evl[j].elapsed_time(evl[j + 1]))
-    moga_ms = call_ms["moga_group_attn"]
+    moga_ms = call_ms[CALLS[2]]   # moga_group_attn, or the combined call
     torch.cuda.synchronize()
     clocks = sampler.stop()
     moga.device_status()
@@ -586,28 +601,34 @@ def run_ours(args):
     fl_stga = stga_flops(wl)
     pk, pk_kind = peaks()
     moga_avg_s = statistics.mean(moga_ms) / 1000.0
-    achieved = fl_moga / moga_avg_s / 1e12
+    # the combined call runs all three branches: its FLOPs are MoGA + STGA
+    fl_call = fl_moga + fl_stga if args.combined else fl_moga
+    achieved = fl_call / moga_avg_s / 1e12
     # a kernel timed inside a timed region of seconds runs under the power
     # cap: the sustained peak applies; a short region gets the burst peak
     sustained = job_ms > 1000.0
     peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
-    traffic, traffic_src = call_traffic(wl)
+    traffic, traffic_src = call_traffic(wl) if not args.combined else (None, "not captured for the combined call")
+    stga_tf = None if args.combined else fl_stga / (statistics.median(call_ms[CALLS[3]]) / 1000.0) / 1e12
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": job_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded counter-based generator; no dataset)",
         "config": config_dict(wl),
         "roofline": {"bound": "tensor",
-                     "kernel": "moga_group_attn call = gather3_kernel (segment-order copy) + attn_kernel<128>",
+                     "kernel": ("visual_attn_branches call = gather_both_kernel + attn_kernel<128> (MoGA, window, "
+                                "frame launches)") if args.combined else
+                               "moga_group_attn call = gather3_kernel (segment-order copy) + attn_kernel<128>",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_kind": "%s %s dense bf16" % (pk_kind, "sustained" if sustained else "burst"),
                      "frac_of_burst": achieved / pk["bf16_tflops"],
                      "traffic": traffic, "traffic_source": traffic_src,
-                     "flops_per_launch": fl_moga, "launch_ms": moga_avg_s * 1e3},
+                     "flops_per_launch": fl_call, "launch_ms": moga_avg_s * 1e3},
         "layer_tflops": (fl_moga + fl_stga) / (job_ms / args.steps / 1000.0) / 1e12,
         "breakdown_ms": {name: statistics.median(v) for name, v in call_ms.items()},
-        "stga_tflops": fl_stga / (statistics.median(call_ms[CALLS[3]]) / 1000.0) / 1e12,
-        "stga_frac": fl_stga / (statistics.median(call_ms[CALLS[3]]) / 1000.0) / 1e12 / peak,
+        "stga_tflops": stga_tf,
+        "stga_frac": stga_tf / peak if stga_tf is not None else None,
+        "attention_call": "visual_attn_branches (one gather)" if args.combined else "moga_group_attn + stga_attn",
         "group_sizes": {"min": int(counts_h.min()), "max": int(counts_h.max()), "sum_sq": float(np.sum(
             counts_h.astype(np.float64) ** 2))},
         "mean_fused_into_stga": bool(args.fused_mean),
@@ -1076,6 +1097,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the end-to-end leg (host copies), e.g. for a profiler's launch list")
+    ap.add_argument("--combined", action="store_true",
+                    help="run the three attention branches as one visual_attn_branches call (one gather pass)")
     ap.add_argument("--fused-mean", action="store_true",
                     help="run stga_attn_mean (mean inside the STGA frame pass) instead of stga_attn + visual_attn_mean")
     ap.add_argument("--train", action="store_true",

@@ -150,6 +150,22 @@ moga_status moga_permute_noalloc(const int32_t* group_id, int64_t N, int32_t M,
  * Returns 0 for arguments the calls would reject. */
 size_t moga_attn_ws_bytes(int64_t N, int32_t H, int32_t hd);
 
+/* ------------------------------------------- the three branches, one gather --
+ * o_acc = MoGA attention (written) + window-group and per-frame attention
+ * (added): the result of moga_group_attn followed by stga_attn on one
+ * stream, bit for bit (the same kernels on the same data), with one pass
+ * over Q, K, V that writes both the group-order and the window-order copy
+ * instead of two passes that each read Q, K, V.  Arguments as for
+ * moga_group_attn and stga_attn together; N must equal geom's T*h*w.
+ * ws: at least visual_attn_ws_bytes(N, H, hd) bytes (6 * N * H * hd * 2:
+ * both copies), 16-byte aligned.  The layer's mean and loss follow as usual
+ * (visual_attn_mean, moga_balance_loss). */
+size_t visual_attn_ws_bytes(int64_t N, int32_t H, int32_t hd);
+moga_status visual_attn_branches(const void* q, const void* k, const void* v, int64_t N, int32_t H, int32_t hd,
+                                 const int32_t* perm, const int32_t* cu_seqlens, int32_t M, const float* gate_prob,
+                                 const moga_stga_geom* geom, float softmax_scale, float* o_acc,
+                                 void* ws, size_t ws_bytes, void* stream);
+
 /* -------------------------------------------------------- group attention --
  * MoGA attention (note, key designs 1-2): for every group i and head h,
  * full non-causal softmax attention among the tokens perm[cu[i] .. cu[i+1]),

@@ -25,6 +25,7 @@ import torch
 from ._lib import MOGA_BF16, MOGA_F32, MogaError, StgaGeom, check, lib  # noqa: F401
 
 __all__ = ["moga_route", "moga_permute", "moga_group_attn", "stga_attn", "stga_attn_train", "stga_attn_mean",
+           "visual_attn_branches",
            "visual_attn_mean", "moga_balance_loss", "visual_attention_forward", "attn_workspace", "device_status",
            "MogaError", "geom_struct", "visual_attention_forward_train", "visual_attention_backward"]
 
@@ -200,6 +201,32 @@ def stga_attn(q, k, v, geom: dict, softmax_scale: float | None = None, o_acc: to
     ws = attn_workspace(q) if ws is None else ws
     check(lib().stga_attn(_ptr(q), _ptr(k), _ptr(v), H, hd, ctypes.byref(s), scale, _ptr(o_acc), _ptr(ws),
                           ws.numel(), _stream()), "stga_attn")
+    del keep
+    return o_acc
+
+
+def visual_attn_branches(q, k, v, perm, cu_seqlens, gate_prob, M: int, geom: dict,
+                         softmax_scale: float | None = None, o_acc: torch.Tensor | None = None,
+                         ws: torch.Tensor | None = None):
+    """o_acc = MoGA attention (written) + window and frame attention (added), with one
+    gather of Q, K, V into both segment orders; equals moga_group_attn + stga_attn."""
+    N, H, hd = _check_qkv(q, k, v, device=False)
+    _check_geom(geom, N)
+    _need(perm, torch.int32, "perm", 1, (N,), device=False)
+    _need(cu_seqlens, torch.int32, "cu_seqlens", 1, (M + 1,), device=False)
+    _need(gate_prob, torch.float32, "gate_prob", 1, (N,), device=False)
+    if o_acc is not None:
+        _need(o_acc, torch.float32, "o_acc", 3, (N, H, hd), device=False)
+    _on_device(q=q, k=k, v=v, perm=perm, cu_seqlens=cu_seqlens, gate_prob=gate_prob, o_acc=o_acc, ws=ws)
+    if o_acc is None:
+        o_acc = torch.empty((N, H, hd), dtype=torch.float32, device=q.device)
+    scale = 1.0 / math.sqrt(hd) if softmax_scale is None else softmax_scale
+    if ws is None:
+        ws = torch.empty(lib().visual_attn_ws_bytes(N, H, hd), dtype=torch.uint8, device=q.device)
+    s, keep = geom_struct(geom)
+    check(lib().visual_attn_branches(_ptr(q), _ptr(k), _ptr(v), N, H, hd, _ptr(perm), _ptr(cu_seqlens), M,
+                                     _ptr(gate_prob), ctypes.byref(s), scale, _ptr(o_acc), _ptr(ws), ws.numel(),
+                                     _stream()), "visual_attn_branches")
     del keep
     return o_acc
 

@@ -33,6 +33,9 @@ SIGNATURES = {
     "moga_group_attn": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I32, _P, _P, _I32, _P, _F32, _P, _P, _SZ, _P]),
     "stga_attn": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _P, _F32, _P, _P, _SZ, _P]),
     "stga_attn_mean": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _P, _F32, _P, _P, _P, _SZ, _P]),
+    "visual_attn_ws_bytes": (_SZ, [_I64, _I32, _I32]),
+    "visual_attn_branches": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I32, _P, _P, _I32, _P, _P, _F32, _P, _P, _SZ,
+                                            _P]),
     "visual_attn_mean": (ctypes.c_int, [_P, _I64, _P, _P]),
     "moga_balance_loss": (ctypes.c_int, [_P, _P, _I64, _I32, _F32, _P, _P]),
     "moga_permute_batched_ws_bytes": (_SZ, [_I64, _I32, _I32]),

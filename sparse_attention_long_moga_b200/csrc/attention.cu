@@ -287,6 +287,46 @@ gather3_kernel(const __grid_constant__ Params p, const uint4* __restrict__ q, co
   }
 }
 
+// Position of token t in the window-major order: the inverse of window_token.
+__host__ __device__ __forceinline__ int window_pos(const Params& p, int t) {
+  const int frame = t / p.hw;
+  const int r = t - frame * p.hw;
+  const int row = r / p.w, col = r - row * p.w;
+  const int win = (row / p.win_h) * p.n_wx + col / p.win_w;
+  const int local = (row % p.win_h) * p.win_w + col % p.win_w;
+  return (win * p.T + frame) * p.whw + local;
+}
+
+// Both segment orders in one pass: for group position j, the token
+// t = perm[j]'s rows of Q, K, V are read once and written to position j of
+// the group-order copy and to position window_pos(t) of the window-order
+// copy (one warp per position).
+__global__ void __launch_bounds__(256)
+gather_both_kernel(const __grid_constant__ Params p, const uint4* __restrict__ q, const uint4* __restrict__ k,
+                   const uint4* __restrict__ v, uint4* __restrict__ gq, uint4* __restrict__ gk, uint4* __restrict__ gv,
+                   uint4* __restrict__ wq, uint4* __restrict__ wk, uint4* __restrict__ wv, int row_u4) {
+  const int j = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (j >= p.N) return;
+  const int lane = threadIdx.x & 31;
+  const int src = __ldg(p.perm + j);
+  if (kCheckIndices && (unsigned)src >= (unsigned)p.N) {
+    if (lane == 0) record_device_error(MOGA_ERR_BAD_INDEX);
+    return;
+  }
+  const size_t so = (size_t)src * row_u4, go = (size_t)j * row_u4, wo = (size_t)window_pos(p, src) * row_u4;
+  for (int c = lane; c < row_u4; c += 32) {
+    const uint4 a = __ldg(q + so + c);
+    const uint4 b = __ldg(k + so + c);
+    const uint4 e = __ldg(v + so + c);
+    gq[go + c] = a;
+    gk[go + c] = b;
+    gv[go + c] = e;
+    wq[wo + c] = a;
+    wk[wo + c] = b;
+    wv[wo + c] = e;
+  }
+}
+
 // ------------------------------------------------------------------ shared memory
 
 template <int HD>
@@ -1000,6 +1040,59 @@ extern "C" moga_status stga_attn_mean(const void* q, const void* k, const void* 
   if (!out) return fail(MOGA_ERR_INVALID_ARG, "stga_attn_mean: null out");
   return stga_impl(q, k, v, H, hd, geom, softmax_scale, o_acc, o_acc, nullptr, nullptr, false, out, ws, ws_bytes,
                    stream, "stga_attn_mean");
+}
+
+// The three branches into one accumulator with a single gather pass:
+// o_acc = MoGA (written), then windows and frames (added), as
+// moga_group_attn followed by stga_attn on one stream, bit for bit.  The
+// workspace holds both copies: [group order: Q, K, V][window order: Q, K, V].
+extern "C" size_t visual_attn_ws_bytes(int64_t N, int32_t H, int32_t hd) {
+  if (N <= 0 || H <= 0 || (hd != 64 && hd != 128) || N * (int64_t)H >= INT32_MAX) return 0;
+  return 2 * attn_ws_bytes(N, H, hd);
+}
+
+extern "C" moga_status visual_attn_branches(const void* q, const void* k, const void* v, int64_t N, int32_t H,
+                                            int32_t hd, const int32_t* perm, const int32_t* cu_seqlens, int32_t M,
+                                            const float* gate_prob, const moga_stga_geom* geom, float softmax_scale,
+                                            float* o_acc, void* ws, size_t ws_bytes, void* stream) {
+  const char* who = "visual_attn_branches";
+  Params prm;
+  int64_t n_geom = 0;
+  moga_status st = stga_params(geom, H, softmax_scale, prm, n_geom, who);
+  if (st != MOGA_OK) return st;
+  if (n_geom != N) return fail(MOGA_ERR_INVALID_ARG, "%s: geometry has %lld tokens, N=%lld", who, (long long)n_geom,
+                               (long long)N);
+  if ((st = check_common(q, k, v, N, H, hd, o_acc, ws, ws_bytes, true, who)) != MOGA_OK) return st;
+  if (ws_bytes < 2 * attn_ws_bytes(N, H, hd))
+    return fail(MOGA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", who, ws_bytes, 2 * attn_ws_bytes(N, H, hd));
+  if (!perm || !cu_seqlens || !gate_prob) return fail(MOGA_ERR_INVALID_ARG, "%s: null pointer", who);
+  if (M < 1 || M > 32) return fail(MOGA_ERR_INVALID_ARG, "%s: M=%d not in [1, 32]", who, M);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = (size_t)N * H * hd * 2;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint8_t* wwin = w + 3 * bytes;
+  prm.perm = perm;
+  prm.cu = cu_seqlens;
+  prm.M = M;
+  prm.gate = gate_prob;
+  prm.o_acc = o_acc;
+  const int row_u4 = H * hd / 8;
+  gather_both_kernel<<<ceil_div((int)N, 8), 256, 0, s>>>(
+      prm, static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v),
+      reinterpret_cast<uint4*>(w), reinterpret_cast<uint4*>(w + bytes), reinterpret_cast<uint4*>(w + 2 * bytes),
+      reinterpret_cast<uint4*>(wwin), reinterpret_cast<uint4*>(wwin + bytes),
+      reinterpret_cast<uint4*>(wwin + 2 * bytes), row_u4);
+  if ((st = check_launch("visual_attn_branches/gather")) != MOGA_OK) return st;
+  // MoGA groups (written), as moga_group_attn
+  prm.mode = MODE_MOGA;
+  const int tiles = (ceil_div((int)N, 2 * BM) + M) * H;
+  if ((st = dispatch_attn(prm, tiles, hd, w, w + bytes, w + 2 * bytes, s)) != MOGA_OK) return st;
+  // windows and frames (added), as stga_attn
+  prm.mode = MODE_WINDOW;
+  if ((st = dispatch_attn(prm, prm.tg_tiles[prm.n_tg], hd, wwin, wwin + bytes, wwin + 2 * bytes, s)) != MOGA_OK)
+    return st;
+  prm.mode = MODE_FRAME;
+  return dispatch_attn(prm, prm.T * H * ceil_div(prm.hw, 2 * BM), hd, q, k, v, s);
 }
 
 // Test hook (declared in include/moga_testing.h): the temporal groups the

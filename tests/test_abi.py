@@ -122,6 +122,24 @@ def test_version(lib):
     assert b"checking" not in lib.moga_version()
 
 
+def test_branches_workspace_and_argument_checks(lib):
+    assert lib.visual_attn_ws_bytes(1000, 4, 128) == 2 * lib.moga_attn_ws_bytes(1000, 4, 128)
+    assert lib.visual_attn_ws_bytes(1000, 4, 96) == 0
+    shots = (ctypes.c_int32 * 2)(2, 2)
+    g = _lib.StgaGeom(4, 4, 8, 2, 4, 2, ctypes.cast(shots, ctypes.POINTER(ctypes.c_int32)), 0, 2)
+    p = ctypes.c_void_p(4096)
+    N, H, hd = 128, 2, 128
+    small = lib.moga_attn_ws_bytes(N, H, hd)
+    # a workspace for one copy only is refused before any launch
+    st = lib.visual_attn_branches(p, p, p, N, H, hd, p, p, 3, p, ctypes.byref(g), ctypes.c_float(0.1), p, p, small,
+                                  None)
+    assert st == 3 and b"workspace" in lib.moga_last_error()
+    # N must be the geometry's token count
+    st = lib.visual_attn_branches(p, p, p, N + 1, H, hd, p, p, 3, p, ctypes.byref(g), ctypes.c_float(0.1), p, p,
+                                  2 * small, None)
+    assert st == 1 and b"geometry" in lib.moga_last_error()
+
+
 def test_status_codes_match_header():
     text = open(HEADER).read()
     enum = dict((n, int(v)) for n, v in re.findall(r"(MOGA_OK|MOGA_ERR_\w+)\s*=\s*(\d+)", text))

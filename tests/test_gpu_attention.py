@@ -55,6 +55,10 @@ def _run_gpu(case, q_scale=1.0):
     o_win, _, o_frame, _ = moga.stga_attn_train(t["q"], t["k"], t["v"], case.geom)
     # the accumulating call adds exactly the values the split call writes
     assert torch.equal(o_static, (torch.zeros_like(o_win) + o_win) + o_frame), case.wl.name
+    # the three branches with one gather pass: the same bits as the two calls
+    o_two = moga.stga_attn(t["q"], t["k"], t["v"], case.geom, o_acc=o_moga.clone())
+    o_one = moga.visual_attn_branches(t["q"], t["k"], t["v"], perm, cu, gate, case.wl.M, case.geom)
+    assert torch.equal(o_one, o_two), case.wl.name
     res = moga.visual_attention_forward(t["x"], t["w_r"], t["bias"], t["q"], t["k"], t["v"], case.wl.M,
                                         case.geom, case.wl.alpha)
     res_unfused = moga.visual_attention_forward(t["x"], t["w_r"], t["bias"], t["q"], t["k"], t["v"], case.wl.M,

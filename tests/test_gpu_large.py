@@ -79,6 +79,13 @@ def test_full_size_sampled(wl, cuda_device):
     moga.device_status()
     # the accumulating call adds the very values the split call writes
     assert _equal_chunked(acc, lambda sl: (o[sl] + o_win[sl]) + o_frame[sl]), wl.name
+    # the three branches with one gather pass give the same bits
+    del ws
+    one = moga.visual_attn_branches(q, k, v, perm, cu, gate, wl.M, geom)
+    moga.device_status()
+    assert _equal_chunked(acc, lambda sl: one[sl]), wl.name
+    del one
+    ws = moga.attn_workspace(q)
 
     g, p_g, p = _route_all(wl, redraw, x_st)
     del x_st
