@@ -340,10 +340,13 @@ struct SmemLayout {
   static constexpr int kNumBars = 24;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kTable = kMisc + 64;
-  static constexpr int kEnd = kTable + (int)sizeof(GroupTable);
+  // epilogue staging: per softmax warp, its 32 rows x 32 fp32 columns (4 KB)
+  static constexpr int kStage = (kTable + (int)sizeof(GroupTable) + 127) & ~127;
+  static constexpr int kStageWarpBytes = 32 * 32 * 4;
+  static constexpr int kEnd = kStage + 8 * kStageWarpBytes;
   // 1 KB slack to align the dynamic base to 1024 bytes; the hd = 64 layout is
   // padded so that two CTAs never share an SM (each holds all 512 TMEM columns)
-  static constexpr int kBytes = (HD == 64 ? 120 * 1024 : kEnd) + 1024;
+  static constexpr int kBytes = (HD == 64 && kEnd < 120 * 1024 ? 120 * 1024 : kEnd) + 1024;
 };
 
 enum Bar : int {
@@ -502,20 +505,36 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
           tc_mma_ts(tmem_o[qt], tmem_s[qt] + ks * 8, bd, idesc_pv, (acc || ks > 0) ? 1u : 0u);
         }
       };
-      bool ok = true;
-      for (int i = 0, L = blockIdx.x; ok; ++i, L += gridDim.x) {
-        const Tile t = decode_tile(p, gt, L);
-        if (!t.valid) break;
+      // The first S product of a tile's query tile 0 is issued right after
+      // the previous tile's last P.V of query tile 0 (the order inside a
+      // tile), when the new Q and K are already there; otherwise, and for
+      // query tile 1 (whose S columns hold the previous tile's last P until
+      // its P.V), after the previous tile's last P.V products.  O_FULL of each
+      // query tile is committed right after its last P.V, so its epilogue
+      // overlaps the other query tile's last products.
+      auto first_s0 = [&](int i, int cc) {
+        if (!(mbar_wait(bar(B_FULL_Q), i & 1, abort_flag, timeout) &&
+              mbar_wait(bar(B_FULL_K + (cc & 1)), (cc >> 1) & 1, abort_flag, timeout)))
+          return false;
+        tc_fence_after();
+        issue_s(0, cc);
+        return true;
+      };
+      auto first_s1 = [&](const Tile& t, int cc) {
+        if (t.q_begin + BM < t.q_end) issue_s(1, cc);
+        if (t.kv_end - t.kv_begin <= BN) tc_commit(bar(B_EMPTY_Q));   // a single K/V tile: Q is read
+        tc_commit(bar(B_EMPTY_K + (cc & 1)));
+      };
+      int L = blockIdx.x;
+      Tile t = decode_tile(p, gt, L);
+      bool ok = t.valid && first_s0(0, c);
+      if (ok) first_s1(t, c);
+      for (int i = 0; ok && t.valid; ++i) {
         const bool has_q1 = t.q_begin + BM < t.q_end;
         const int nq = has_q1 ? 2 : 1;
         const int n_kv = ceil_div(t.kv_end - t.kv_begin, BN);
-        ok = mbar_wait(bar(B_FULL_Q), i & 1, abort_flag, timeout) &&
-             mbar_wait(bar(B_FULL_K + (c & 1)), (c >> 1) & 1, abort_flag, timeout);
-        if (!ok) break;
-        tc_fence_after();
-        for (int qt = 0; qt < nq; ++qt) issue_s(qt, c);
-        if (n_kv == 1) tc_commit(bar(B_EMPTY_Q));
-        tc_commit(bar(B_EMPTY_K + (c & 1)));
+        const Tile tn = decode_tile(p, gt, L + gridDim.x);
+        bool next_started = false;
         for (int j = 0; j < n_kv; ++j, ++c) {
           const int st = c & 1;
           const uint32_t ph = (c >> 1) & 1;
@@ -529,10 +548,18 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
             tc_fence_after();
             issue_pv(qt, c, j > 0);
             ++pc[qt];
+            if (!more) {
+              tc_commit(bar(B_O_FULL + qt));
+              ++oc[qt];
+            }
             if (qt == 0 && more) {
               if (!(ok = mbar_wait(bar(B_FULL_K + ((c + 1) & 1)), ((c + 1) >> 1) & 1, abort_flag, timeout))) break;
               tc_fence_after();
               issue_s(0, c + 1);
+            } else if (qt == 0 && tn.valid && has_q1 && mbar_test(bar(B_FULL_Q), (i + 1) & 1) &&
+                       mbar_test(bar(B_FULL_K + ((c + 1) & 1)), ((c + 1) >> 1) & 1)) {
+              if (!(ok = first_s0(i + 1, c + 1))) break;
+              next_started = true;
             }
           }
           if (!ok) break;
@@ -544,10 +571,12 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
           }
         }
         if (!ok) break;
-        for (int qt = 0; qt < nq; ++qt) {
-          tc_commit(bar(B_O_FULL + qt));
-          ++oc[qt];
+        if (tn.valid) {
+          if (!next_started) ok = first_s0(i + 1, c);
+          if (ok) first_s1(tn, c);
         }
+        t = tn;
+        L += gridDim.x;
       }
       // every MMA issued here has finished before TMEM is released
       tc_commit(bar(B_MMA_END));
@@ -667,16 +696,50 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
       mbar_arrive(bar(B_O_EMPTY + qt));   // O may be overwritten by the next tile now
       const int q_idx = t.q_begin + qt * BM + row;
       const int tok = q_idx < t.q_end ? token_of(p, q_idx) : -1;
-      if (tok >= 0) {
-        float scale = 1.0f / l_run;
-        if (p.mode == MODE_MOGA) scale *= __ldg(p.gate + tok);
-        float4* d4 = reinterpret_cast<float4*>(p.o_acc + ((size_t)tok * p.H + t.head) * HD);
-        if (p.lse != nullptr) p.lse[(size_t)tok * p.H + t.head] = m_run + log2f(l_run);
-        if (p.mode == MODE_MOGA || p.write_static) {
+      float scale = 1.0f / l_run;
+      if (tok >= 0 && p.mode == MODE_MOGA) scale *= __ldg(p.gate + tok);
+      if (tok >= 0 && p.lse != nullptr) p.lse[(size_t)tok * p.H + t.head] = m_run + log2f(l_run);
+      if (p.out == nullptr || p.mode == MODE_MOGA || p.write_static) {
+        // Rows leave through shared memory so that each warp instruction
+        // writes whole 128-byte lines: per 32-column chunk, every thread puts
+        // its row there (16-byte chunk k of row r at slot k ^ (r & 7), which
+        // keeps the stores and the loads free of bank conflicts), then the
+        // warp writes four rows per instruction, eight lanes per row.  The
+        // MoGA branch stores; the static branches add into the accumulator
+        // with fire-and-forget vector reductions (each element is updated by
+        // exactly one thread per launch, so the result equals load-add-store
+        // without the load latency).
+        float4* stage = reinterpret_cast<float4*>(smem + S::kStage + warp * S::kStageWarpBytes);
+        const bool plain = p.mode == MODE_MOGA || p.write_static;
+        const int sub = lane & 7;
 #pragma unroll
-          for (int e = 0; e < HD / 4; ++e)
-            d4[e] = make_float4(o[4 * e] * scale, o[4 * e + 1] * scale, o[4 * e + 2] * scale, o[4 * e + 3] * scale);
-        } else if (p.out != nullptr) {
+        for (int cc = 0; cc < HD / 32; ++cc) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            stage[lane * 8 + (k ^ (lane & 7))] =
+                make_float4(o[cc * 32 + 4 * k] * scale, o[cc * 32 + 4 * k + 1] * scale, o[cc * 32 + 4 * k + 2] * scale,
+                            o[cc * 32 + 4 * k + 3] * scale);
+          __syncwarp();
+#pragma unroll
+          for (int r4 = 0; r4 < 8; ++r4) {
+            const int rr = r4 * 4 + (lane >> 3);   // row of this warp written by this lane
+            const int tr = __shfl_sync(0xffffffffu, tok, rr);
+            const float4 val = stage[rr * 8 + (sub ^ (rr & 7))];
+            if (tr >= 0) {
+              float4* d = reinterpret_cast<float4*>(p.o_acc + ((size_t)tr * p.H + t.head) * HD + cc * 32) + sub;
+              if (plain)
+                *d = val;
+              else
+                asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(d), "f"(val.x), "f"(val.y),
+                             "f"(val.z), "f"(val.w)
+                             : "memory");
+            }
+          }
+          __syncwarp();
+        }
+      } else if (tok >= 0) {
+        const float4* d4 = reinterpret_cast<const float4*>(p.o_acc + ((size_t)tok * p.H + t.head) * HD);
+        {
           // last branch of the layer: the three-way mean, fused (the frames
           // partition the tokens, so this thread owns the row)
           // product and sum rounded separately (no FMA contraction), as in
@@ -690,16 +753,6 @@ attn_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMa
             dst[e] = make_uint4(pack_bf16x2(avg(a.x, oe[0]), avg(a.y, oe[1])), pack_bf16x2(avg(a.z, oe[2]), avg(a.w, oe[3])),
                                 pack_bf16x2(avg(b.x, oe[4]), avg(b.y, oe[5])), pack_bf16x2(avg(b.z, oe[6]), avg(b.w, oe[7])));
           }
-        } else {
-          // the static branches add into the accumulator with fire-and-forget
-          // vector reductions (each element is updated by exactly one thread
-          // per launch, so the result is the same as load-add-store, without
-          // the load latency in the epilogue)
-#pragma unroll
-          for (int e = 0; e < HD / 4; ++e)
-            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(d4 + e), "f"(o[4 * e] * scale),
-                         "f"(o[4 * e + 1] * scale), "f"(o[4 * e + 2] * scale), "f"(o[4 * e + 3] * scale)
-                         : "memory");
         }
       }
     }
