@@ -48,22 +48,24 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # current kernels: gather3_kernel<0> 302.06 + 259.95 MB, attn_kernel<128>
 # (MoGA launch) 304.74 + 158.97 MB.  Set to None whenever either kernel
 # changes, until it is captured again.
-CALL_TRAFFIC_BYTES = 1.0293e9
-CALL_TRAFFIC_UNITS = 32760 * 12 * 128
-CALL_TRAFFIC_SOURCE = "ncu dram__bytes_read.sum + dram__bytes_write.sum, gather3_kernel<0> + attn_kernel<128> MoGA launch"
+# DRAM bytes (ncu dram__bytes_read.sum + dram__bytes_write.sum) of one launch
+# each, captured on the 32,760-token workload (12 heads, hd 128)
+TRAFFIC_UNITS = 32760 * 12 * 128
+KERNEL_TRAFFIC_BYTES = 306173952 + 161697792            # attn_kernel<128>, MoGA launch
+CALL_TRAFFIC_BYTES = KERNEL_TRAFFIC_BYTES + 302057472 + 259337472   # + gather3_kernel<0>
 
 
-def call_traffic(wl):
-    """DRAM bytes of one moga_group_attn call: the captured figure, scaled by
-    the Q/K/V elements processed for another workload (the copy moves every
-    element once and each group's K/V stays L2-resident while its tiles run)."""
-    if CALL_TRAFFIC_BYTES is None:
-        return None, "not captured for the current kernels"
+def scaled_traffic(wl, captured, what):
+    """DRAM bytes of one launch (or call) on this workload: the captured
+    figure, scaled by the Q/K/V elements processed for another workload (the
+    copy moves every element once; the attention launch reads Q, K, V once,
+    each group's K/V staying L2-resident while its tiles run, and writes the
+    output once)."""
+    src = "ncu dram__bytes_read.sum + dram__bytes_write.sum, " + what
     units = wl.N * wl.H * wl.hd
-    if units == CALL_TRAFFIC_UNITS:
-        return CALL_TRAFFIC_BYTES, CALL_TRAFFIC_SOURCE + " (captured on this workload)"
-    return CALL_TRAFFIC_BYTES * units / CALL_TRAFFIC_UNITS, (
-        CALL_TRAFFIC_SOURCE + ", captured on the 32,760-token workload and scaled by N*H*hd")
+    if units == TRAFFIC_UNITS:
+        return captured, src + " (captured on this workload)"
+    return captured * units / TRAFFIC_UNITS, src + ", captured on the 32,760-token workload and scaled by N*H*hd"
 
 
 def peaks():
@@ -513,6 +515,19 @@ def run_ours(args):
     else:
         CALLS = ("route", "permute", "moga_group_attn", "stga_attn_mean", "moga_balance_loss")
     evl = [torch.cuda.Event(enable_timing=True) for _ in range(len(CALLS) + 1)]
+    # the attention launches alone, without their gather copies: the library
+    # records these events around the attention-kernel launches of a call
+    attn_calls = CALLS[2:3] if args.combined else CALLS[2:4]
+    hook = L.moga_test_set_attn_events
+    hook.restype = None
+    hook.argtypes = [moga.ctypes.c_void_p, moga.ctypes.c_void_p]
+    kev = {name: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)] for name in attn_calls}
+    for pairs in kev.values():
+        for a, b in pairs:   # creates the handles
+            a.record(stream)
+            b.record(stream)
+    t_index = [0]
 
     def step(xd, qd, kd, vd, timed=False, out=out, loss=loss):
         c = moga.check
@@ -520,6 +535,14 @@ def run_ours(args):
         def mark(i):
             if timed:
                 evl[i].record(stream)
+
+        def arm(name):
+            if timed:
+                hook(*kev[name][t_index[0]])
+
+        def disarm():
+            if timed:
+                hook(None, None)
         mark(0)
         c(L.moga_route(P(xd), P(w_r), moga.MOGA_BF16, P(bias) if bias is not None else None, N, wl.d, M, P(g),
                        P(gate), P(rws), rws.numel(), sp), "route")
@@ -528,26 +551,33 @@ def run_ours(args):
         mark(2)
         if args.combined:
             # the three branches with one gather of Q, K, V into both orders
+            arm(CALLS[2])
             c(L.visual_attn_branches(P(qd), P(kd), P(vd), N, H, hd, P(perm), P(cu), M, P(gate),
                                      moga.ctypes.byref(gs), scale, P(o_acc), P(aws), aws.numel(), sp), "branches")
+            disarm()
             mark(3)
             c(L.visual_attn_mean(P(o_acc), o_acc.numel(), P(out), sp), "mean")
             mark(len(CALLS) - 1)
             c(L.moga_balance_loss(P(counts), P(rws), N, M, wl.alpha, P(loss), sp), "loss")
             mark(len(CALLS))
             return
+        arm(CALLS[2])
         c(L.moga_group_attn(P(qd), P(kd), P(vd), N, H, hd, P(perm), P(cu), M, P(gate), scale, P(o_acc), P(aws),
                             aws.numel(), sp), "moga")
+        disarm()
         mark(3)
+        arm(CALLS[3])
         if not args.fused_mean:
             c(L.stga_attn(P(qd), P(kd), P(vd), H, hd, moga.ctypes.byref(gs), scale, P(o_acc), P(aws), aws.numel(),
                           sp), "stga")
+            disarm()
             mark(4)
             c(L.visual_attn_mean(P(o_acc), o_acc.numel(), P(out), sp), "mean")
         else:
             # the three-way mean taken inside the frame pass of STGA
             c(L.stga_attn_mean(P(qd), P(kd), P(vd), H, hd, moga.ctypes.byref(gs), scale, P(o_acc), P(out), P(aws),
                                aws.numel(), sp), "stga_mean")
+            disarm()
         mark(len(CALLS) - 1)
         c(L.moga_balance_loss(P(counts), P(rws), N, M, wl.alpha, P(loss), sp), "loss")
         mark(len(CALLS))
@@ -575,13 +605,16 @@ def run_ours(args):
     sampler.start()
     for i in range(args.steps):
         flush.zero_()
+        t_index[0] = i
         evs[i][0].record(stream)
         step(x, q, k, v, timed=True)
         evs[i][1].record(stream)
         evl[-1].synchronize()
         for j, name in enumerate(CALLS):
             call_ms[name].append(evl[j].elapsed_time(evl[j + 1]))
+    kern_ms = {name: [a.elapsed_time(b) for a, b in pairs] for name, pairs in kev.items()}
     moga_ms = call_ms[CALLS[2]]   # moga_group_attn, or the combined call
+    moga_kern_ms = kern_ms[CALLS[2]]
     torch.cuda.synchronize()
     clocks = sampler.stop()
     moga.device_status()
@@ -601,33 +634,52 @@ def run_ours(args):
     fl_stga = stga_flops(wl)
     pk, pk_kind = peaks()
     moga_avg_s = statistics.mean(moga_ms) / 1000.0
+    kern_avg_s = statistics.mean(moga_kern_ms) / 1000.0
     # the combined call runs all three branches: its FLOPs are MoGA + STGA
     fl_call = fl_moga + fl_stga if args.combined else fl_moga
-    achieved = fl_call / moga_avg_s / 1e12
+    achieved = fl_call / kern_avg_s / 1e12
+    call_achieved = fl_call / moga_avg_s / 1e12
     # a kernel timed inside a timed region of seconds runs under the power
     # cap: the sustained peak applies; a short region gets the burst peak
     sustained = job_ms > 1000.0
     peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
-    traffic, traffic_src = call_traffic(wl) if not args.combined else (None, "not captured for the combined call")
-    stga_tf = None if args.combined else fl_stga / (statistics.median(call_ms[CALLS[3]]) / 1000.0) / 1e12
+    if args.combined:
+        traffic, traffic_src = None, "not captured for the combined call"
+        call_traffic, call_traffic_src = None, traffic_src
+    else:
+        traffic, traffic_src = scaled_traffic(wl, KERNEL_TRAFFIC_BYTES, "attn_kernel<128> MoGA launch")
+        call_traffic, call_traffic_src = scaled_traffic(wl, CALL_TRAFFIC_BYTES,
+                                                        "gather3_kernel<0> + attn_kernel<128> MoGA launch")
+    stga_tf = stga_call_tf = None
+    if not args.combined:
+        stga_tf = fl_stga / (statistics.median(kern_ms[CALLS[3]]) / 1000.0) / 1e12
+        stga_call_tf = fl_stga / (statistics.median(call_ms[CALLS[3]]) / 1000.0) / 1e12
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": job_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded counter-based generator; no dataset)",
         "config": config_dict(wl),
         "roofline": {"bound": "tensor",
-                     "kernel": ("visual_attn_branches call = gather_both_kernel + attn_kernel<128> (MoGA, window, "
-                                "frame launches)") if args.combined else
-                               "moga_group_attn call = gather3_kernel (segment-order copy) + attn_kernel<128>",
+                     "kernel": ("attn_kernel<128>: the MoGA, window and frame launches of visual_attn_branches"
+                                if args.combined else "attn_kernel<128>: the MoGA launch of moga_group_attn"),
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_kind": "%s %s dense bf16" % (pk_kind, "sustained" if sustained else "burst"),
                      "frac_of_burst": achieved / pk["bf16_tflops"],
                      "traffic": traffic, "traffic_source": traffic_src,
-                     "flops_per_launch": fl_call, "launch_ms": moga_avg_s * 1e3},
+                     "flops_per_launch": fl_call, "launch_ms": kern_avg_s * 1e3,
+                     "timing": "CUDA events recorded by the library around the attention launch(es) of each "
+                               "timed call, on the launching stream"},
+        "attention_call_roofline": {
+            "call": ("visual_attn_branches = gather_both_kernel + attn_kernel<128> x 3" if args.combined else
+                     "moga_group_attn = gather3_kernel<0> (segment-order copy) + attn_kernel<128>"),
+            "achieved": call_achieved, "frac": call_achieved / peak, "frac_of_burst": call_achieved / pk["bf16_tflops"],
+            "call_ms": moga_avg_s * 1e3, "traffic": call_traffic, "traffic_source": call_traffic_src},
         "layer_tflops": (fl_moga + fl_stga) / (job_ms / args.steps / 1000.0) / 1e12,
         "breakdown_ms": {name: statistics.median(v) for name, v in call_ms.items()},
+        "attention_kernels_ms": {name: statistics.median(v) for name, v in kern_ms.items()},
         "stga_tflops": stga_tf,
         "stga_frac": stga_tf / peak if stga_tf is not None else None,
+        "stga_call_tflops": stga_call_tf,
         "attention_call": "visual_attn_branches (one gather)" if args.combined else "moga_group_attn + stga_attn",
         "group_sizes": {"min": int(counts_h.min()), "max": int(counts_h.max()), "sum_sq": float(np.sum(
             counts_h.astype(np.float64) ** 2))},

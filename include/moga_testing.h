@@ -11,6 +11,17 @@
  *   memory and exits (no trap, no hang).  moga_device_status() reports it.
  * Pass (0, 0) to restore normal operation.
  *
+ * moga_test_set_attn_events(before, after) takes two cudaEvent_t handles
+ * (created by the caller, on the device of the calls) for the calling host
+ * thread: the next forward attention-kernel launch of moga_group_attn,
+ * stga_attn, stga_attn_mean, visual_attn_branches or their batched forms
+ * records `before` on its stream just in front of it, and every attention-
+ * kernel launch from then on records `after` just behind it, so that after
+ * one call the two events bracket that call's attention launches without
+ * its gather copies.  Set it again before each call to be timed; (NULL,
+ * NULL) switches it off.  A failed record returns MOGA_ERR_CUDA from the
+ * call.  Profiling use only: it changes no result.
+ *
  * moga_test_stga_groups(geom, out, cap) validates geom as stga_attn does and
  * returns the number n of temporal groups its launches use (-1 if stga_attn
  * would reject the geometry; moga_last_error() says why), writing for group
@@ -49,6 +60,7 @@ extern "C" {
 #endif
 
 void moga_test_set_attn_debug(long long timeout_cycles, int flags);
+void moga_test_set_attn_events(void* before, void* after);
 int32_t moga_test_stga_groups(const moga_stga_geom* geom, int32_t* out, int32_t cap);
 int32_t moga_test_attn_tiles(int32_t mode, const int32_t* cu_seqlens, int32_t M, int64_t N, int32_t H,
                              const moga_stga_geom* geom, int32_t* out, int32_t cap);

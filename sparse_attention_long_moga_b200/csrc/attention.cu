@@ -839,12 +839,34 @@ static int sm_count() {
   return n > 0 ? n : 148;
 }
 
+// Timing hook (declared in include/moga_testing.h): events recorded on the
+// launching stream around the attention-kernel launches of the next call on
+// this thread.  armed 1: `before` goes in front of the next launch; armed 2:
+// `after` follows every launch until the hook is set again.
+static thread_local cudaEvent_t t_ev_before = nullptr, t_ev_after = nullptr;
+static thread_local int t_ev_armed = 0;
+extern "C" void moga_test_set_attn_events(void* before, void* after) {
+  t_ev_before = static_cast<cudaEvent_t>(before);
+  t_ev_after = static_cast<cudaEvent_t>(after);
+  t_ev_armed = (before && after) ? 1 : 0;
+}
+
 // `tiles` is the number of tile pairs (or an upper bound); the persistent
 // grid has one CTA per SM at most.
 static moga_status dispatch_attn(const Params& prm, int tiles, int hd, const void* q, const void* k, const void* v,
                                  cudaStream_t s) {
   const int grid = std::min(tiles, sm_count());
-  return hd == 128 ? launch_attn<128>(prm, grid, q, k, v, s) : launch_attn<64>(prm, grid, q, k, v, s);
+  if (t_ev_armed == 1) {
+    const cudaError_t e = cudaEventRecord(t_ev_before, s);
+    if (e != cudaSuccess) return fail(MOGA_ERR_CUDA, "attention timing event: %s", cudaGetErrorString(e));
+    t_ev_armed = 2;
+  }
+  const moga_status st = hd == 128 ? launch_attn<128>(prm, grid, q, k, v, s) : launch_attn<64>(prm, grid, q, k, v, s);
+  if (st == MOGA_OK && t_ev_armed == 2) {
+    const cudaError_t e = cudaEventRecord(t_ev_after, s);
+    if (e != cudaSuccess) return fail(MOGA_ERR_CUDA, "attention timing event: %s", cudaGetErrorString(e));
+  }
+  return st;
 }
 
 static size_t attn_ws_bytes(int64_t N, int H, int hd) { return 3 * (size_t)N * H * hd * 2; }

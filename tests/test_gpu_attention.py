@@ -36,6 +36,12 @@ SMALL = {
                                    tg_max=0, win_h=7, win_w=3, aug=1),
     "mid_2shot": W.Workload("mid_2shot", T=6, h=10, w=20, d=64, H=2, hd=128, M=3, shots=(4, 2), tg_max=3,
                             win_h=5, win_w=10),
+    # more work tiles than SMs, so every persistent CTA runs several tiles and
+    # crosses tile boundaries (single key tiles; then tiles of one or two
+    # query tiles over two to four key tiles)
+    "many_tiles_M32_H40": EDGE.with_(name="edge_M32_H40", M=32, H=40),
+    "many_tiles_M3_H64": W.Workload("mid_H64", T=6, h=10, w=20, d=64, H=64, hd=128, M=3, shots=(4, 2), tg_max=3,
+                                    win_h=5, win_w=10),
 }
 
 
@@ -153,3 +159,35 @@ def test_sampled_rows_full_size(wl, cuda_device):
             got[n].append(res[n][toks, h])
     for n in got:
         assert_close(np.concatenate(got[n]), np.concatenate(ref[n]), "%s sampled %s" % (n, wl.name))
+
+
+def test_attention_timing_hook(cuda_device):
+    """moga_test_set_attn_events brackets the attention launch of one call (not
+    its gather copy), changes no result, and records nothing once switched off."""
+    import ctypes
+    import torch
+    import sparse_attention_long_moga_b200 as moga
+    case = Case(SMALL["many_tiles_M3_H64"])
+    t = case.gpu()
+    g, gate, _ = moga.moga_route(t["x"], t["w_r"], t["bias"])
+    perm, cu, _, _ = moga.moga_permute(g, case.wl.M)
+    hook = moga._lib.lib().moga_test_set_attn_events
+    hook.restype = None
+    hook.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    ref = moga.moga_group_attn(t["q"], t["k"], t["v"], perm, cu, gate, case.wl.M)
+    a, b, c0, c1 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
+    a.record()
+    b.record()
+    c0.record()
+    hook(a, b)
+    got = moga.moga_group_attn(t["q"], t["k"], t["v"], perm, cu, gate, case.wl.M)
+    hook(None, None)
+    c1.record()
+    c1.synchronize()
+    moga.device_status()
+    assert torch.equal(got, ref)
+    k_ms, c_ms = a.elapsed_time(b), c0.elapsed_time(c1)
+    assert 0.0 < k_ms <= c_ms
+    moga.moga_group_attn(t["q"], t["k"], t["v"], perm, cu, gate, case.wl.M)
+    torch.cuda.synchronize()
+    assert a.elapsed_time(b) == k_ms

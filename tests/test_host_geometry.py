@@ -97,7 +97,7 @@ def test_testing_header_symbols_are_exported(groups_fn):
     lib, _ = groups_fn
     text = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "moga_testing.h")).read(), flags=re.S)
     names = re.findall(r"^\s*(?:void|int32_t)\s+(\w+)\s*\(", text, flags=re.M)
-    assert set(names) == {"moga_test_set_attn_debug", "moga_test_stga_groups", "moga_test_attn_tiles",
-                          "moga_test_window_tokens", "moga_test_bwd_units"}
+    assert set(names) == {"moga_test_set_attn_debug", "moga_test_set_attn_events", "moga_test_stga_groups",
+                          "moga_test_attn_tiles", "moga_test_window_tokens", "moga_test_bwd_units"}
     for name in names:
         assert hasattr(lib, name)
