@@ -13,6 +13,8 @@
 //                    picked through perm for MoGA, through the window map for
 //                    the static windows), so that every group is a contiguous
 //                    row range.  Frames are contiguous already and skip it.
+//                    (gather_both_kernel writes both orders in one pass for
+//                    the call that runs all three branches.)
 //   attn_kernel      one CTA per (group, head, pair of 128-row query tiles):
 //     warps 0-3 / 4-7  softmax + epilogue of query tile 0 / 1
 //                      (thread = query row = TMEM lane)
@@ -24,7 +26,11 @@
 //   The softmax writes P as bf16 pairs over the first 64 columns of its S
 //   and the P.V product reads it from there (A operand in tensor memory).
 //   Issue order per KV tile j:  PV0_j, S0_{j+1}, PV1_j, S1_{j+1}, so the
-//   softmax of one tile runs while the tensor core serves the other.
+//   softmax of one tile runs while the tensor core serves the other; the
+//   same order continues across work tiles (the next tile's first S0 goes
+//   between the last PV0 and PV1 when its Q and K have landed).
+//   Output rows leave through a per-warp shared-memory stage as whole
+//   128-byte lines.
 //   The running row max only moves (and O is rescaled) when it grows by
 //   more than 2^8; the final 1/l uses the same reference, so the result is
 //   exact.
