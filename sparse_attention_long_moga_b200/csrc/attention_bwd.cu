@@ -247,16 +247,38 @@ __device__ __forceinline__ uint32_t bwd_pack(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// fp32 gradient rows added into dst[token][head][:] (fire-and-forget vector
-// reductions; keys shared by two window groups receive two contributions)
+// fp32 gradient rows g (this lane's row; tok < 0: none) added into
+// dst[token][head][:] with fire-and-forget vector reductions (keys shared by
+// two window groups receive two contributions).  Called by all 32 lanes of a
+// warp: per 32-column chunk each lane puts its row into the warp's 4 KB
+// stage (16-byte chunk k of row r at slot k ^ (r & 7), free of bank
+// conflicts), then each reduction covers four rows of 128 bytes, eight lanes
+// per row, instead of 32 scattered rows.
 template <int HD>
-__device__ __forceinline__ void add_rows(float* dst, int tok, int H, int head, const float* g) {
-  float4* d4 = reinterpret_cast<float4*>(dst + ((size_t)tok * H + head) * HD);
+__device__ __forceinline__ void add_rows(float* dst, int tok, int H, int head, const float* g, float4* stage,
+                                         int lane) {
+  const int sub = lane & 7;
 #pragma unroll
-  for (int e = 0; e < HD / 4; ++e)
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(d4 + e), "f"(g[4 * e]), "f"(g[4 * e + 1]),
-                 "f"(g[4 * e + 2]), "f"(g[4 * e + 3])
-                 : "memory");
+  for (int cc = 0; cc < HD / 32; ++cc) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      stage[lane * 8 + (k ^ (lane & 7))] =
+          make_float4(g[cc * 32 + 4 * k], g[cc * 32 + 4 * k + 1], g[cc * 32 + 4 * k + 2], g[cc * 32 + 4 * k + 3]);
+    __syncwarp();
+#pragma unroll
+    for (int r4 = 0; r4 < 8; ++r4) {
+      const int rr = r4 * 4 + (lane >> 3);   // row of this warp written by this lane
+      const int tr = __shfl_sync(0xffffffffu, tok, rr);
+      const float4 v = stage[rr * 8 + (sub ^ (rr & 7))];
+      if (tr >= 0) {
+        float4* d = reinterpret_cast<float4*>(dst + ((size_t)tr * H + head) * HD + cc * 32) + sub;
+        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(d), "f"(v.x), "f"(v.y), "f"(v.z),
+                     "f"(v.w)
+                     : "memory");
+      }
+    }
+    __syncwarp();
+  }
 }
 
 // Common prologue of both kernels: barriers, group table, TMEM (512 columns).
@@ -553,7 +575,9 @@ bwd_dkdv_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUt
         if (part == 1)
 #pragma unroll
           for (int e = 0; e < HD; ++e) g[e] *= b.scale;   // dK = scale dS^T Q
-        if (tok >= 0) add_rows<HD>(part == 0 ? b.dv : b.dk, tok, p.H, u.head, g);
+        // the streamed stages are idle once every product has finished
+        add_rows<HD>(part == 0 ? b.dv : b.dk, tok, p.H, u.head, g,
+                     reinterpret_cast<float4*>(smem + SM::kStageA + warp * 4096), lane);
       }
     }
   }
@@ -700,7 +724,8 @@ bwd_dq_kernel(const __grid_constant__ BwdParams b, const __grid_constant__ CUten
 #pragma unroll
       for (int e = 0; e < HD; ++e) g[e] *= b.scale;   // dQ = scale dS K
       const int tok = in ? token_of(p, qr) : -1;
-      if (tok >= 0) add_rows<HD>(b.dq, tok, p.H, u.head, g);
+      // the streamed stages are idle once every product has finished
+      add_rows<HD>(b.dq, tok, p.H, u.head, g, reinterpret_cast<float4*>(smem + SM::kStageA + warp * 4096), lane);
     }
   }
   bwd_teardown<HD>(tmem);
