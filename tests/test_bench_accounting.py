@@ -68,3 +68,28 @@ def test_cpu_baseline_row_costs_match_flop_count(wl):
     cost_tok = counts[g] + kv_win + wl.hw
     flops_from_rows = 4.0 * wl.hd * float(cost_tok.sum()) * wl.H
     assert flops_from_rows == bench.moga_flops(counts, wl.H, wl.hd) + bench.stga_flops(wl)
+
+
+def test_traffic_figures_scale_with_the_elements_moved():
+    """`roofline.traffic` is the attention launch's captured DRAM bytes, the
+    call's figure adds its gather copy; both are per launch on the captured
+    workload and proportional to N * H * hd elsewhere."""
+    wl = W.resolved(W.WAN13B_5S)
+    kern, src = bench.scaled_traffic(wl, bench.KERNEL_TRAFFIC_BYTES, "kernel")
+    call, _ = bench.scaled_traffic(wl, bench.CALL_TRAFFIC_BYTES, "call")
+    assert "captured on this workload" in src
+    assert (kern, call) == (bench.KERNEL_TRAFFIC_BYTES, bench.CALL_TRAFFIC_BYTES)
+    # the gather copy reads and writes Q, K, V once: it sits between the
+    # algorithmic bytes of one read + one write of Q, K, V (2 x 302 MB) and
+    # the copy's written bytes alone
+    gather = call - kern
+    qkv = 3 * wl.N * wl.H * wl.hd * 2
+    assert qkv < gather <= 2 * qkv
+    # the attention launch reads Q, K, V once and writes the fp32 output at
+    # most once: its traffic stays within the algorithmic bytes' band
+    alg = 4 * wl.N * wl.H * wl.hd * 2 + 4 * wl.N
+    assert 1.0 <= kern / alg < 1.5
+    big = W.resolved(W.LONG_60S)
+    k2, src2 = bench.scaled_traffic(big, bench.KERNEL_TRAFFIC_BYTES, "kernel")
+    assert "scaled by N*H*hd" in src2
+    assert k2 == pytest.approx(kern * (big.N * big.H * big.hd) / (wl.N * wl.H * wl.hd), rel=1e-12)
