@@ -20,6 +20,8 @@ CASES = [
     W.TINY,
     W.WAN13B_5S,
     W.MULTISHOT_10S,
+    W.WAN14B_30S_M5,
+    W.LONG_60S,   # the benchmark's headline workload: ten shots, borrowed frames at nine cuts
     # a middle shot shorter than the borrowed-frame count, temporal groups of 2
     W.Workload("acct_short_shot", T=5, h=6, w=10, d=64, H=3, hd=128, M=7, shots=(2, 1, 2), tg_max=2, win_h=3,
                win_w=5),
